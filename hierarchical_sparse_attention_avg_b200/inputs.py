@@ -1,0 +1,52 @@
+"""Seeded synthetic inputs for the Lighthouse layer.
+
+This module only draws random numbers; it holds none of the layer's arithmetic.  Both the CUDA path's tests and
+benchmark and the CPU oracle's tests take their inputs from here, so both sides see the same bytes.
+
+Recipe (the value distributions of the long-context configurations): every token row of Q, K and V is
+``bf16(s * z)`` with ``z ~ N(0, 1)^d`` and one factor ``s = exp(0.5 * n)``, ``n ~ N(0, 1)`` (lognormal(0, 0.5)) per
+row; the upstream gradient is ``bf16(N(0, 1))``.  Draws come from one ``torch.Generator`` seeded with ``seed`` on the
+requested device, in the order Q, K, V, dO.  CPU and CUDA generators give different (but each reproducible) bytes.
+"""
+
+from __future__ import annotations
+
+import torch
+
+
+def _generator(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _scaled_rows(shape, g, device) -> torch.Tensor:
+    z = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    n = torch.randn(shape[:-1] + (1,), generator=g, device=device, dtype=torch.float32)
+    z.mul_(torch.exp(0.5 * n))
+    return z.to(torch.bfloat16)
+
+
+def make_inputs(B: int, H: int, N: int, d: int, seed: int = 0, device="cpu", with_grad: bool = True):
+    """Return ``(q, k, v, dout)`` bf16 tensors of shape ``[B, H, N, d]`` (``dout`` is None without grad)."""
+    g = _generator(seed, device)
+    shape = (B, H, N, d)
+    q = _scaled_rows(shape, g, device)
+    k = _scaled_rows(shape, g, device)
+    v = _scaled_rows(shape, g, device)
+    dout = None
+    if with_grad:
+        dout = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return q, k, v, dout
+
+
+def make_scores(B: int, H: int, rows: int, seed: int = 0, device="cpu", ties: bool = False) -> torch.Tensor:
+    """Non-negative fp32 scores ``[B, H, rows]`` for feeding the top-K step directly.
+
+    With ``ties=True`` the values are drawn from a small set so that many scores are equal, which exercises the
+    lower-index tie rule."""
+    g = _generator(seed, device)
+    if ties:
+        return torch.randint(0, 4, (B, H, rows), generator=g, device=device).to(torch.float32)
+    z = torch.randn((B, H, rows), generator=g, device=device, dtype=torch.float32)
+    return z * z
