@@ -1,0 +1,328 @@
+"""Benchmark of the Lighthouse selection-and-attend layer: forward + backward tokens/s on one B200 per rank.
+
+One step = ``lh_forward`` + ``lh_backward`` (pool, score, top-K, gather, causal attention, scatter and their
+backward) over one batch of synthetic inputs resident in HBM.  Multi-GPU runs are weak-scaled replicas (each rank
+its own batch, no collective on the data path); the step time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "tiny4K": dict(B=1, H=2, N=4096, d=64, L=3, p=4, k=256, C=8),
+    "train32K": dict(B=1, H=16, N=32768, d=64, L=4, p=4, k=2048, C=16),
+    "ctx98K": dict(B=1, H=16, N=98304, d=64, L=4, p=4, k=2048, C=16),
+    "long512K": dict(B=1, H=16, N=524288, d=128, L=4, p=4, k=4096, C=32),
+    "stress1M": dict(B=1, H=8, N=1048576, d=128, L=4, p=4, k=4096, C=32),
+}
+DEFAULT_WORKLOAD = "long512K"
+METRIC = "Lighthouse fwd+bwd tokens/s at N=512K; HBM GB/s and attention TFLOP/s vs peak"
+UNIT = "tokens/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm=pk["hbm_gbs"], bf16=pk["bf16_tflops"], bf16_sust=pk["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def kernel_work(w: dict) -> dict:
+    """Algorithmic bytes (HBM-bound kernels) or FLOPs (attention) of ONE launch of each kernel, all heads."""
+    B, H, N, d, L, p, k = w["B"], w["H"], w["N"], w["d"], w["L"], w["p"], w["k"]
+    BH = B * H
+    Nl = [N // p ** lev for lev in range(L)]
+    kl = [min(k, Nl[lev]) if lev < L - 1 else Nl[lev] for lev in range(L)]
+    S = sum(kl)
+    R, Rs = sum(Nl), sum(Nl[:-1])
+    row = d * 2
+    # rows of the raw input that selected entries below the coarsest level cover (read by the gather)
+    gather_src = sum(kl[lev] * p ** lev for lev in range(L - 1)) + Nl[-1]
+    partial = sum(Nl[lev] for lev in range(L - 1) if kl[lev] < Nl[lev])
+    return {
+        "pool_score": ("hbm", BH * (3 * N * row + 3 * Nl[-1] * row + Rs * 4)),
+        "topk": ("hbm", BH * (partial * 4 * 2 + sum(kl[:-1]) * 4)),
+        "order": ("hbm", BH * (S * 4 * 2 + sum(kl[:-1]) * 4)),
+        "gather": ("hbm", BH * 3 * (gather_src + S) * row),
+        "attn_fwd": ("tensor", 2.0 * S * S * d * BH),
+        "scatter": ("hbm", BH * (N * row + S * row + R * 4)),
+        "scatter_bwd": ("hbm", BH * (N * row + 2 * S * row + S * 4 + S * d * 4)),
+        "attn_bwd": ("tensor", 5.0 * S * S * d * BH),
+        "unpool_bwd": ("hbm", BH * (3 * N * row + S * d * 4 + 2 * S * row + R * 4)),
+    }, S
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def cpu_baseline(w: dict, seed: int = 0) -> dict:
+    """The CPU oracle timed on one head of the workload (forward + backward), scaled to tokens/s of the whole
+    workload (heads are independent, so the time of all B*H heads is B*H times one head's)."""
+    from oracle import lighthouse as O
+    from hierarchical_sparse_attention_avg_b200.inputs import make_inputs
+
+    q, k, v, dout = make_inputs(1, 1, w["N"], w["d"], seed=seed, device="cpu")
+    f = lambda t: t[0, 0].float().numpy().astype(np.float64)
+    qf, kf, vf, df = f(q), f(k), f(v), f(dout)
+    P = O.Params(1, 1, w["N"], w["d"], w["L"], w["p"], w["k"], w["C"])
+    t0 = time.perf_counter()
+    fwd = O.forward_head(qf, kf, vf, P)
+    O.backward_head(df, fwd, P)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    heads = w["B"] * w["H"]
+    return {"value": w["B"] * w["N"] / (dt * heads), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"1 of {heads} heads of {w_name(w)} (forward+backward, {dt:.1f} s), scaled by {heads}",
+            "seconds": dt}
+
+
+def w_name(w):
+    for n, v in WORKLOADS.items():
+        if v == w:
+            return n
+    return "custom"
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(w)
+    times = [cpu_baseline(w)["seconds"] for _ in range(args.steps)]
+    heads = w["B"] * w["H"]
+    sec = sum(times) / len(times)
+    value = w["B"] * w["N"] / (sec * heads)
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+            "warmup": min(args.warmup, 1), "ms_per_step": sec * 1e3 * heads, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w_name(w), **w, "sample": "one head per step, scaled by B*H"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"one head of {heads} per step (forward+backward), scaled by {heads}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from hierarchical_sparse_attention_avg_b200 import lh
+    from hierarchical_sparse_attention_avg_b200.inputs import make_inputs
+
+    P = lh.Params(**w)
+    q, k, v, dout = make_inputs(w["B"], w["H"], w["N"], w["d"], seed=rank, device=dev)
+    o = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ctx = lh.new_ctx(P, dev)
+    ws = lh.new_workspace(P, dev)
+
+    def step():
+        lh.lh_forward(P, q, k, v, o=o, ctx=ctx, ws=ws)
+        lh.lh_backward(P, dout, ctx, dq=dq, dk=dk, dv=dv, ws=ws)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    lh.lh_profile_enable(True)
+    lh.lh_profile_read()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    lh.lh_profile_enable(False)
+    prof = lh.lh_profile_read()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    status = lh.lh_get_status(dev)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {lh.error_string(status)}")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w["B"] * w["N"] * world
+    value = tokens / (ms / 1e3)
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs, the step, D2H of its outputs
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, dout)]
+        host_out = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
+        dev_in = (q, k, v, dout)
+        dev_out = (o, dq, dk, dv)
+
+        def e2e_step():
+            for h, d_ in zip(host_in, dev_in):
+                d_.copy_(h, non_blocking=True)
+            step()
+            for h, d_ in zip(host_out, dev_out):
+                h.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(1, min(args.steps, 3))
+        if world > 1:
+            torch.distributed.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = a0.elapsed_time(a1) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = sum(t.numel() * t.element_size() for t in host_in)
+        obytes = sum(t.numel() * t.element_size() for t in host_out)
+        e2e = {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+               "d2h_bytes_per_step": obytes, "ms_per_step": ms_e2e, "steps": n_e2e}
+
+    peaks = load_peaks()
+    work, S = kernel_work(w)
+    total_kernel_ms = sum(v_[1] for v_ in prof.values()) or 1.0
+    kernels = {}
+    for name, (launches, kms) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
+        bound, amount = work.get(name, ("hbm", 0))
+        per_ms = kms / launches
+        if bound == "tensor":
+            ach = amount / (per_ms / 1e3) / 1e12
+            kernels[name] = {"launches": launches, "ms": per_ms, "share": kms / total_kernel_ms, "bound": "tensor",
+                             "achieved": ach, "unit": "TFLOP/s", "frac": ach / peaks["bf16_sust"]}
+        else:
+            ach = amount / (per_ms / 1e3) / 1e9
+            kernels[name] = {"launches": launches, "ms": per_ms, "share": kms / total_kernel_ms, "bound": "hbm",
+                             "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm"]}
+    top = max(kernels.items(), key=lambda kv: kv[1]["share"])
+    tname, tk = top
+    roofline = {"kernel": tname, "bound": tk["bound"], "achieved": tk["achieved"],
+                "peak": peaks["bf16_sust"] if tk["bound"] == "tensor" else peaks["hbm"], "unit": tk["unit"],
+                "frac": tk["frac"], "traffic": None,
+                "peak_source": f"{peaks['src']} ({'bf16 sustained' if tk['bound'] == 'tensor' else 'HBM copy'})"}
+    gpu_launches = sum(v_[0] for v_ in prof.values())
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, **w, "S": S, "parallelism": f"replicas{world}",
+                           "l2": "inputs larger than L2 (2 GB per tensor), no flush"
+                           if w["B"] * w["H"] * w["N"] * w["d"] * 2 > 126e6 else "inputs smaller than L2, no flush"},
+                "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
+                "clocks": clk, "e2e": e2e}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = {k_: v_ for k_, v_ in cpu_baseline(w).items() if k_ != "seconds"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,462 @@
+// api.cu — the C ABI of liblh.so: argument validation, size queries, buffer layouts and the launch sequences
+// of the step-wise and fused entry points.  Semantics of every entry point are documented in include/lh.h.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace lh {
+
+__device__ int g_lh_status = 0;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Fill the size table; returns LH_OK, LH_ERR_INVALID_ARG or LH_ERR_UNSUPPORTED.
+int make_dims(const lh_params* P, LhDims* dm) {
+  if (!P) return LH_ERR_INVALID_ARG;
+  memset(dm, 0, sizeof(*dm));
+  if (P->B < 1 || P->H < 1 || P->N < 1 || P->d < 1 || P->L < 1 || P->p < 2 || P->k < 1 || P->C < 1 ||
+      P->flags != 0 || P->L > LH_MAX_LEVELS)
+    return LH_ERR_INVALID_ARG;
+  int64_t w = 1;
+  for (int l = 1; l < P->L; ++l) {
+    w *= P->p;
+    if (w > P->N) return LH_ERR_INVALID_ARG;
+  }
+  if (P->N % w) return LH_ERR_INVALID_ARG;
+  dm->B = P->B; dm->H = P->H; dm->N = P->N; dm->d = P->d; dm->L = P->L; dm->p = P->p; dm->k = P->k; dm->C = P->C;
+  const int64_t BH = (int64_t)P->B * P->H;
+  int64_t S = 0, R = 0, Rs = 0, Rp = 0;
+  int nPartial = 0;
+  int64_t wl = 1;
+  for (int l = 0; l < P->L; ++l) {
+    const int64_t n = P->N / wl;
+    dm->Nl[l] = (int)n;
+    dm->wl[l] = (int)wl;
+    dm->off[l] = (int)R;
+    if (l >= 1) dm->poff[l] = (int)Rp;
+    int64_t kl = n;
+    if (l <= P->L - 2 && P->k < n) {
+      if (n % P->C || P->k % P->C) return LH_ERR_INVALID_ARG;
+      kl = P->k;
+      if (l != nPartial) return LH_ERR_INVALID_ARG;  // unreachable: level sizes decrease
+      dm->seloff[l] = nPartial * P->k;
+      ++nPartial;
+    }
+    dm->kl[l] = (int)kl;
+    S += kl;
+    R += n;
+    if (l <= P->L - 2) Rs += n;
+    if (l >= 1) Rp += n;
+    wl *= P->p;
+  }
+  dm->BH = (int)BH;
+  dm->S = (int)S;
+  dm->R = (int)R;
+  dm->Rs = (int)Rs;
+  dm->Rp = (int)Rp;
+  dm->nPartial = nPartial;
+  dm->Ksel = nPartial * P->k;
+  // what the kernels are built for
+  if (P->d != 64 && P->d != 128) return LH_ERR_UNSUPPORTED;
+  if (P->p != 2 && P->p != 4 && P->p != 8) return LH_ERR_UNSUPPORTED;
+  if (P->L > 5 || w > 512) return LH_ERR_UNSUPPORTED;
+  if (nPartial > 0 && P->k / P->C > 512) return LH_ERR_UNSUPPORTED;
+  if (BH > 65535 || R > INT32_MAX / 2) return LH_ERR_UNSUPPORTED;
+  return LH_OK;
+}
+
+struct CtxLayout {
+  size_t qg, kg, vg, og, lse, idx_g, slot, total;
+};
+CtxLayout ctx_layout(const LhDims& dm) {
+  CtxLayout c;
+  const size_t rows = (size_t)dm.BH * dm.S;
+  size_t o = 0;
+  c.qg = o; o = align_up(o + rows * dm.d * 2);
+  c.kg = o; o = align_up(o + rows * dm.d * 2);
+  c.vg = o; o = align_up(o + rows * dm.d * 2);
+  c.og = o; o = align_up(o + rows * dm.d * 2);
+  c.lse = o; o = align_up(o + rows * 4);
+  c.idx_g = o; o = align_up(o + rows * 4);
+  c.slot = o; o = align_up(o + (size_t)dm.BH * dm.R * 4);
+  c.total = o;
+  return c;
+}
+
+struct WsLayout {
+  // forward / selection
+  size_t scores, coarse[3], sel, fwd_total;
+  // backward
+  size_t dog, dvec, dqacc, dkg, dvg, bwd_total;
+  size_t total;
+};
+WsLayout ws_layout(const LhDims& dm) {
+  WsLayout w;
+  size_t o = 0;
+  w.scores = o; o = align_up(o + (size_t)dm.BH * dm.Rs * 4);
+  const size_t coarse = (size_t)dm.BH * dm.Nl[dm.L - 1] * dm.d * 2;
+  for (int i = 0; i < 3; ++i) { w.coarse[i] = o; o = align_up(o + coarse); }
+  w.sel = o; o = align_up(o + (size_t)dm.BH * dm.Ksel * 4);
+  w.fwd_total = o;
+  const size_t rows = (size_t)dm.BH * dm.S;
+  o = 0;
+  w.dog = o; o = align_up(o + rows * dm.d * 2);
+  w.dvec = o; o = align_up(o + rows * 4);
+  w.dqacc = o; o = align_up(o + rows * dm.d * 4);
+  w.dkg = o; o = align_up(o + rows * dm.d * 2);
+  w.dvg = o; o = align_up(o + rows * dm.d * 2);
+  w.bwd_total = o;
+  w.total = w.fwd_total > w.bwd_total ? w.fwd_total : w.bwd_total;
+  if (w.total == 0) w.total = kAlign;
+  return w;
+}
+
+inline bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+// Device status word of the current device.
+int status_ptr(int** out) {
+  static std::mutex mu;
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LH_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lh_status) != cudaSuccess) return LH_ERR_CUDA;
+    cache[dev] = static_cast<int*>(p);
+  }
+  *out = cache[dev];
+  return LH_OK;
+}
+
+int prepare(const lh_params* P, LhDims* dm) {
+  int rc = make_dims(P, dm);
+  if (rc) return rc;
+  return status_ptr(&dm->status);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+int make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LH_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)bh};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
+}
+
+}  // namespace lh
+
+using namespace lh;
+
+#define LH_TRY(expr)        \
+  do {                      \
+    const int rc_ = (expr); \
+    if (rc_) return rc_;    \
+  } while (0)
+
+extern "C" {
+
+const char* lh_error_string(int status) {
+  switch (status) {
+    case LH_OK: return "ok";
+    case LH_ERR_INVALID_ARG: return "invalid argument";
+    case LH_ERR_UNSUPPORTED: return "unsupported shape";
+    case LH_ERR_CUDA: return "CUDA error";
+    case LH_ERR_TIMEOUT: return "device wait timed out";
+    case LH_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int lh_validate(const lh_params* P) {
+  LhDims dm;
+  return make_dims(P, &dm);
+}
+
+int64_t lh_S(const lh_params* P) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  return (rc == LH_OK || rc == LH_ERR_UNSUPPORTED) ? dm.S : -1;
+}
+
+int64_t lh_level_size(const lh_params* P, int level) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  if ((rc != LH_OK && rc != LH_ERR_UNSUPPORTED) || level < 0 || level >= dm.L) return -1;
+  return dm.Nl[level];
+}
+
+int64_t lh_level_offset(const lh_params* P, int level) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  if ((rc != LH_OK && rc != LH_ERR_UNSUPPORTED) || level < 0 || level >= dm.L) return -1;
+  return dm.off[level];
+}
+
+int64_t lh_pyramid_rows(const lh_params* P) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  return (rc == LH_OK || rc == LH_ERR_UNSUPPORTED) ? dm.Rp : -1;
+}
+
+int64_t lh_score_rows(const lh_params* P) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  return (rc == LH_OK || rc == LH_ERR_UNSUPPORTED) ? dm.Rs : -1;
+}
+
+int64_t lh_slot_rows(const lh_params* P) {
+  LhDims dm;
+  const int rc = make_dims(P, &dm);
+  return (rc == LH_OK || rc == LH_ERR_UNSUPPORTED) ? dm.R : -1;
+}
+
+size_t lh_ctx_bytes(const lh_params* P) {
+  LhDims dm;
+  if (make_dims(P, &dm) != LH_OK) return 0;
+  return ctx_layout(dm).total;
+}
+
+int lh_ctx_layout(const lh_params* P, lh_ctx_layout_t* out) {
+  LhDims dm;
+  LH_TRY(make_dims(P, &dm));
+  if (!out) return LH_ERR_INVALID_ARG;
+  const CtxLayout c = ctx_layout(dm);
+  out->qg = c.qg; out->kg = c.kg; out->vg = c.vg; out->og = c.og;
+  out->lse = c.lse; out->idx_g = c.idx_g; out->slot = c.slot; out->total = c.total;
+  return LH_OK;
+}
+
+size_t lh_workspace_bytes(const lh_params* P) {
+  LhDims dm;
+  if (make_dims(P, &dm) != LH_OK) return 0;
+  return ws_layout(dm).total;
+}
+
+int lh_pool(const lh_params* P, const void* x, void* pyr, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  if (dm.L == 1) return LH_OK;
+  if (!aligned16(x) || !aligned16(pyr)) return LH_ERR_INVALID_ARG;
+  PoolJobs jobs;
+  memset(&jobs, 0, sizeof(jobs));
+  PoolJob& j = jobs.job[0];
+  j.x = x;
+  j.pyr = pyr;
+  j.pyr_rows = dm.Rp;
+  for (int l = 1; l < dm.L; ++l) {
+    j.write_mask |= 1u << l;
+    j.row_off[l] = dm.poff[l];
+  }
+  return launch_pool_score(jobs, 1, dm, (cudaStream_t)stream);
+}
+
+int lh_score_topk(const lh_params* P, const void* k, const float* scores_in, float* scores_out, int32_t* idx_g,
+                  int32_t* slot, void* ws, size_t ws_bytes, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(idx_g) || !aligned16(slot)) return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const float* scores = scores_in;
+  if (dm.L >= 2 && !scores_in) {
+    if (!aligned16(k) || (scores_out && !aligned16(scores_out))) return LH_ERR_INVALID_ARG;
+    float* dst = scores_out ? scores_out : reinterpret_cast<float*>(wsb + w.scores);
+    PoolJobs jobs;
+    memset(&jobs, 0, sizeof(jobs));
+    jobs.job[0].x = k;
+    jobs.job[0].scores = dst;
+    LH_TRY(launch_pool_score(jobs, 1, dm, st));
+    scores = dst;
+  } else if (dm.L >= 2 && !aligned16(scores_in)) {
+    return LH_ERR_INVALID_ARG;
+  }
+  int32_t* sel = reinterpret_cast<int32_t*>(wsb + w.sel);
+  LH_TRY(launch_topk(scores, sel, slot, dm, st));
+  return launch_order(sel, idx_g, slot, dm, st);
+}
+
+int lh_gather(const lh_params* P, const void* q, const void* k, const void* v, const void* q_pyr, const void* k_pyr,
+              const void* v_pyr, const int32_t* idx_g, void* qg, void* kg, void* vg, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  const void* xs[3] = {q, k, v};
+  const void* ps[3] = {q_pyr, k_pyr, v_pyr};
+  void* outs[3] = {qg, kg, vg};
+  GatherJobs jobs;
+  memset(&jobs, 0, sizeof(jobs));
+  if (!aligned16(idx_g)) return LH_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i) {
+    if (!aligned16(xs[i]) || !aligned16(outs[i])) return LH_ERR_INVALID_ARG;
+    if (dm.L > 1 && !aligned16(ps[i])) return LH_ERR_INVALID_ARG;
+    GatherJob& j = jobs.job[i];
+    j.x = xs[i];
+    j.pyr = ps[i];
+    j.pyr_rows = dm.Rp;
+    for (int l = 1; l < dm.L; ++l) {
+      j.pyr_mask |= 1u << l;
+      j.row_off[l] = dm.poff[l];
+    }
+    j.out = outs[i];
+  }
+  return launch_gather(jobs, 3, idx_g, dm, (cudaStream_t)stream);
+}
+
+int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, void* og, float* lse,
+              void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  if (!aligned16(qg) || !aligned16(kg) || !aligned16(vg) || !aligned16(og) || !aligned16(lse))
+    return LH_ERR_INVALID_ARG;
+  return launch_attn_fwd(qg, kg, vg, og, lse, dm, (cudaStream_t)stream);
+}
+
+int lh_scatter(const lh_params* P, const void* og, const int32_t* slot, void* o, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  if (!aligned16(og) || !aligned16(slot) || !aligned16(o)) return LH_ERR_INVALID_ARG;
+  return launch_scatter(og, slot, o, dm, (cudaStream_t)stream);
+}
+
+int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, void* o, void* ctx, void* ws,
+               size_t ws_bytes, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ctx))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  const CtxLayout c = ctx_layout(dm);
+  uint8_t* cb = static_cast<uint8_t*>(ctx);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const void* xs[3] = {q, k, v};
+  const int top = dm.L - 1;
+
+  // 1-2: pool Q, K, V in one launch; only the coarsest level is stored, plus the key scores
+  if (dm.L >= 2) {
+    PoolJobs pj;
+    memset(&pj, 0, sizeof(pj));
+    for (int i = 0; i < 3; ++i) {
+      pj.job[i].x = xs[i];
+      pj.job[i].pyr = wsb + w.coarse[i];
+      pj.job[i].pyr_rows = dm.Nl[top];
+      pj.job[i].write_mask = 1u << top;
+      pj.job[i].row_off[top] = 0;
+    }
+    pj.job[1].scores = reinterpret_cast<float*>(wsb + w.scores);
+    LH_TRY(launch_pool_score(pj, 3, dm, st));
+  }
+  // 3: top-K and the gathered order
+  int32_t* idx_g = reinterpret_cast<int32_t*>(cb + c.idx_g);
+  int32_t* slot = reinterpret_cast<int32_t*>(cb + c.slot);
+  int32_t* sel = reinterpret_cast<int32_t*>(wsb + w.sel);
+  LH_TRY(launch_topk(reinterpret_cast<float*>(wsb + w.scores), sel, slot, dm, st));
+  LH_TRY(launch_order(sel, idx_g, slot, dm, st));
+  // 4a: gather (levels 1..L-2 recomputed from the raw rows with the same summation tree)
+  GatherJobs gj;
+  memset(&gj, 0, sizeof(gj));
+  const size_t outs[3] = {c.qg, c.kg, c.vg};
+  for (int i = 0; i < 3; ++i) {
+    gj.job[i].x = xs[i];
+    gj.job[i].pyr = wsb + w.coarse[i];
+    gj.job[i].pyr_rows = dm.Nl[top];
+    gj.job[i].pyr_mask = dm.L >= 2 ? (1u << top) : 0u;
+    gj.job[i].row_off[top] = 0;
+    gj.job[i].out = cb + outs[i];
+  }
+  LH_TRY(launch_gather(gj, 3, idx_g, dm, st));
+  // 4b: attention over the gathered sequence
+  LH_TRY(launch_attn_fwd(cb + c.qg, cb + c.kg, cb + c.vg, cb + c.og, reinterpret_cast<float*>(cb + c.lse), dm, st));
+  // 5: scatter back
+  return launch_scatter(cb + c.og, slot, o, dm, st);
+}
+
+int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq, void* dk, void* dv, void* ws,
+                size_t ws_bytes, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(dout) || !aligned16(ctx) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  const CtxLayout c = ctx_layout(dm);
+  const uint8_t* cb = static_cast<const uint8_t*>(ctx);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const int32_t* idx_g = reinterpret_cast<const int32_t*>(cb + c.idx_g);
+  const int32_t* slot = reinterpret_cast<const int32_t*>(cb + c.slot);
+  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  float* dqacc = reinterpret_cast<float*>(wsb + w.dqacc);
+  LH_TRY(launch_scatter_bwd(dout, idx_g, wsb + w.dog, cb + c.og, dvec, dqacc, dm, st));
+  LH_TRY(launch_attn_bwd(cb + c.qg, cb + c.kg, cb + c.vg, wsb + w.dog, reinterpret_cast<const float*>(cb + c.lse),
+                         dvec, dqacc, wsb + w.dkg, wsb + w.dvg, dm, st));
+  return launch_unpool_bwd(dqacc, wsb + w.dkg, wsb + w.dvg, slot, dq, dk, dv, dm, st);
+}
+
+int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, void* dog, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  if (!aligned16(dout) || !aligned16(idx_g) || !aligned16(dog)) return LH_ERR_INVALID_ARG;
+  return launch_scatter_bwd(dout, idx_g, dog, nullptr, nullptr, nullptr, dm, (cudaStream_t)stream);
+}
+
+int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const void* og,
+                  const float* lse, const void* dog, float* dqg, void* dkg, void* dvg, void* ws, size_t ws_bytes,
+                  void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(qg) || !aligned16(kg) || !aligned16(vg) || !aligned16(og) || !aligned16(lse) || !aligned16(dog) ||
+      !aligned16(dqg) || !aligned16(dkg) || !aligned16(dvg))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  float* dvec = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.dvec);
+  LH_TRY(launch_attn_prep(og, dog, dvec, dqg, dm, st));
+  return launch_attn_bwd(qg, kg, vg, dog, lse, dvec, dqg, dkg, dvg, dm, st);
+}
+
+int lh_get_status(void* stream) {
+  int* p = nullptr;
+  if (status_ptr(&p)) return LH_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LH_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LH_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return LH_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// internal.h — host-side declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lh_common.cuh"
+
+namespace lh {
+
+// One pooling job: one input tensor, optional pyramid output (levels chosen by write_mask, level l written at
+// row row_off[l] of a per-head block of pyr_rows rows), optional score output (levels 0..L-2).
+struct PoolJob {
+  const void* x;
+  void* pyr;
+  int pyr_rows;
+  uint32_t write_mask;  // bit l set: write level l (1 <= l <= L-1)
+  int row_off[LH_MAX_LEVELS];
+  float* scores;        // [BH, Rs] or nullptr
+};
+struct PoolJobs {
+  PoolJob job[3];
+};
+
+// One gather job: rows of one tensor.  Source of level l >= 1: pyr (per-head rows pyr_rows, level l at
+// row_off[l]) when non-null for that level, else recomputed from x.
+struct GatherJob {
+  const void* x;
+  const void* pyr;
+  int pyr_rows;
+  uint32_t pyr_mask;  // bit l set: level l is read from pyr
+  int row_off[LH_MAX_LEVELS];
+  void* out;          // [BH, S, d]
+};
+struct GatherJobs {
+  GatherJob job[3];
+};
+
+int launch_pool_score(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st);
+int launch_gather(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st);
+int launch_topk(const float* scores, int32_t* sel, int32_t* slot, const LhDims& dm, cudaStream_t st);
+int launch_order(const int32_t* sel, int32_t* idx_g, int32_t* slot, const LhDims& dm, cudaStream_t st);
+int launch_scatter(const void* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st);
+// dog[s] = window sum of dout; when og/dvec/dqacc are non-null also dvec[s] = <dog[s], og[s]> and dqacc[s] = 0.
+int launch_scatter_bwd(const void* dout, const int32_t* idx_g, void* dog, const void* og, float* dvec,
+                       float* dqacc, const LhDims& dm, cudaStream_t st);
+int launch_attn_prep(const void* og, const void* dog, float* dvec, float* dqacc, const LhDims& dm, cudaStream_t st);
+int launch_unpool_bwd(const float* dqg, const void* dkg, const void* dvg, const int32_t* slot, void* dq, void* dk,
+                      void* dv, const LhDims& dm, cudaStream_t st);
+int launch_attn_fwd(const void* qg, const void* kg, const void* vg, void* og, float* lse, const LhDims& dm,
+                    cudaStream_t st);
+int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog, const float* lse,
+                    const float* dvec, float* dqacc, void* dkg, void* dvg, const LhDims& dm, cudaStream_t st);
+
+// Encode a 3-D bf16 tensor map over [BH][rows][d] with a {64, 128, 1} box and 128-byte swizzle.
+int make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh);
+
+inline int check_launch() { return cudaGetLastError() == cudaSuccess ? LH_OK : LH_ERR_CUDA; }
+
+// Brackets the kernel launches of its scope with CUDA events on `st` while tracing is enabled
+// (lh_profile_enable); a no-op otherwise.
+class KernelTimer {
+ public:
+  KernelTimer(const char* name, cudaStream_t st);
+  ~KernelTimer();
+
+ private:
+  int slot_ = -1;
+  cudaStream_t st_;
+};
+
+}  // namespace lh

@@ -1,0 +1,249 @@
+// pool_gather.cu — step 1 (symmetric average-pool pyramid), step 2 (per-head l2-norm score) and the row
+// gather of step 4.
+//
+// Pooling follows [W] 核心方法 §1 对称金字塔池化 (Q, K and V average-pooled alike into a multi-level
+// pyramid); scoring follows [W] 核心方法 §2 and [E] "Как four-stage pipeline…" (parameter-free per-head l2
+// norm).  The arithmetic is the one the layer's definition fixes so that results are bit-exact everywhere:
+//   level sums in fp64, each level summing its p children left to right from the first child;
+//   pooled value = bf16_RN(sum / p^l);
+//   score = fp32_RN(sum of squares: 8 left to right per 8-feature group, then a pairwise tree over groups).
+//
+// Thread layout: a "group" of d/8 lanes owns one row, each lane 8 features (one 16-byte vector).  The pairwise
+// tree over the groups of a row is an xor-butterfly over those lanes (float addition is commutative, so every
+// lane ends with the same bits).
+#include "internal.h"
+
+namespace lh {
+
+namespace {
+
+constexpr int kPoolThreads = 256;
+
+__host__ __device__ constexpr int ipow(int b, int e) { return e == 0 ? 1 : b * ipow(b, e - 1); }
+
+__device__ __forceinline__ void load_row8(const uint4& raw, double (&x)[8]) {
+  float f[8];
+  unpack8(raw, f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = (double)f[i];
+}
+
+// Score of one row: squared l2 norm of the (bf16) values x, summed in the fixed order, rounded to fp32.
+template <int G>
+__device__ __forceinline__ float row_score(const double (&x)[8]) {
+  double s = x[0] * x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) s = fma(x[i], x[i], s);  // x*x is exact in fp64: fma == add of the square
+#pragma unroll
+  for (int off = 1; off < G; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  return __double2float_rn(s);
+}
+
+// Round 8 fp64 sums / w to bf16 (single rounding), returning packed bits and the bf16 values as fp64.
+__device__ __forceinline__ uint4 round_pooled(const double (&sum)[8], double inv_w, double (&val)[8]) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    b[i] = f64_to_bf16_bits_rne(sum[i] * inv_w);  // inv_w = 1/p^l is exact for power-of-two p
+    val[i] = (double)__uint_as_float(b[i] << 16);
+  }
+  return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
+}
+
+// One group processes one block of W = P^(L-1) consecutive tokens of one head (one coarsest entry), building
+// every level of the pyramid inside the block in registers.
+template <int D, int P, int L>
+__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, LhDims dm) {
+  constexpr int G = D / 8;
+  constexpr int GPB = kPoolThreads / G;
+  constexpr int W = ipow(P, L - 1);
+  constexpr int TB = (W < 8) ? W : 8;  // tokens loaded per batch (a multiple of P)
+  static_assert(TB % P == 0, "batch must hold whole level-1 entries");
+
+  const PoolJob& job = jobs.job[blockIdx.y];
+  const int lane = threadIdx.x % G;
+  const int64_t group = (int64_t)blockIdx.x * GPB + threadIdx.x / G;
+  const int nblk = dm.N / W;
+  const int64_t total = (int64_t)dm.BH * nblk;
+  const bool active = group < total;
+  const int64_t gi = active ? group : total - 1;  // idle groups shadow a valid one (shuffles need the warp)
+  const int bh = (int)(gi / nblk);
+  const int blk = (int)(gi % nblk);
+
+  const __nv_bfloat16* xrow =
+      reinterpret_cast<const __nv_bfloat16*>(job.x) + ((int64_t)bh * dm.N + (int64_t)blk * W) * D + lane * 8;
+  float* scores = job.scores ? job.scores + (int64_t)bh * dm.Rs : nullptr;
+  __nv_bfloat16* pyr = reinterpret_cast<__nv_bfloat16*>(job.pyr);
+
+  double acc[L][8];  // acc[l]: running sum of the current level-l entry (l >= 1)
+
+#pragma unroll 1
+  for (int t0 = 0; t0 < W; t0 += TB) {
+    uint4 raw[TB];
+#pragma unroll
+    for (int u = 0; u < TB; ++u) raw[u] = ld_stream16(xrow + (int64_t)(t0 + u) * D);
+
+#pragma unroll
+    for (int g1 = 0; g1 < TB / P; ++g1) {
+#pragma unroll
+      for (int c = 0; c < P; ++c) {
+        double x[8];
+        load_row8(raw[g1 * P + c], x);
+        if (scores) {  // level 0 is scored whenever L >= 2
+          float s = row_score<G>(x);
+          if (active && lane == 0) scores[dm.off[0] + (int64_t)blk * W + t0 + g1 * P + c] = s;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[1][i] = (c == 0) ? x[i] : acc[1][i] + x[i];
+      }
+      // level-1 entry complete; walk up while parents complete
+      int jloc = t0 / P + g1;  // index of the completed level-1 entry inside this block
+#pragma unroll
+      for (int lev = 1; lev < L; ++lev) {
+        if (lev > 1) {
+          const int c = jloc % P;  // child index of the completed level-(lev-1) entry
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[lev][i] = (c == 0) ? acc[lev - 1][i] : acc[lev][i] + acc[lev - 1][i];
+          if (c != P - 1) break;
+          jloc /= P;
+        }
+        const int64_t j = (int64_t)blk * (W / ipow(P, lev)) + jloc;  // global index at level lev
+        const bool write = (job.write_mask >> lev) & 1u;
+        const bool score = scores && lev <= L - 2;
+        if (write || score) {
+          double val[8];
+          const uint4 packed = round_pooled(acc[lev], 1.0 / (double)ipow(P, lev), val);
+          if (write && active)
+            st16(pyr + ((int64_t)bh * job.pyr_rows + job.row_off[lev] + j) * D + lane * 8, packed);
+          if (score) {
+            float s = row_score<G>(val);
+            if (active && lane == 0) scores[dm.off[lev] + j] = s;
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int D, int P, int LEV>
+__device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8]) {
+  if constexpr (LEV == 0) {
+    load_row8(ld16(p), out);
+  } else {
+    constexpr int CW = ipow(P, LEV - 1);
+#pragma unroll 1
+    for (int c = 0; c < P; ++c) {
+      double ch[8];
+      tree_sum<D, P, LEV - 1>(p + (int64_t)c * CW * D, ch);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? ch[i] : out[i] + ch[i];
+    }
+  }
+}
+
+// Pooled value of entry (lev, j) recomputed from the raw rows with the same summation tree as the pool kernel.
+template <int D, int P>
+__device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
+  double s[8], val[8];
+  switch (lev) {
+    case 1: tree_sum<D, P, 1>(x0, s); break;
+    case 2: tree_sum<D, P, 2>(x0, s); break;
+    case 3: tree_sum<D, P, 3>(x0, s); break;
+    default: tree_sum<D, P, 4>(x0, s); break;
+  }
+  return round_pooled(s, 1.0 / (double)ipow(P, lev), val);
+}
+
+// One group per gathered row (b, h, s): copy (level 0), read (pyramid) or recompute (pooled) the row.
+template <int D, int P>
+__global__ void __launch_bounds__(256) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
+                                                     LhDims dm) {
+  constexpr int G = D / 8;
+  const GatherJob& job = jobs.job[blockIdx.y];
+  const int lane = threadIdx.x % G;
+  const int64_t row = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
+  if (row >= (int64_t)dm.BH * dm.S) return;
+  const int bh = (int)(row / dm.S);
+  const int gid = idx_g[row];
+  int lev = 0;
+#pragma unroll
+  for (int l = 1; l < LH_MAX_LEVELS; ++l)
+    if (l < dm.L && gid >= dm.off[l]) lev = l;
+  const int j = gid - dm.off[lev];
+  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(job.x);
+  uint4 v;
+  if (lev == 0) {
+    v = ld16(x + ((int64_t)bh * dm.N + j) * D + lane * 8);
+  } else if ((job.pyr_mask >> lev) & 1u) {
+    v = ld16(reinterpret_cast<const __nv_bfloat16*>(job.pyr) +
+             ((int64_t)bh * job.pyr_rows + job.row_off[lev] + j) * D + lane * 8);
+  } else {
+    v = pooled_row<D, P>(x + ((int64_t)bh * dm.N + (int64_t)j * dm.wl[lev]) * D + lane * 8, lev);
+  }
+  st16(reinterpret_cast<__nv_bfloat16*>(job.out) + row * D + lane * 8, v);
+}
+
+template <int D, int P, int L>
+int launch_pool_t(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+  constexpr int G = D / 8;
+  constexpr int W = ipow(P, L - 1);
+  const int64_t groups = (int64_t)dm.BH * (dm.N / W);
+  const int64_t blocks = (groups + kPoolThreads / G - 1) / (kPoolThreads / G);
+  if (blocks > 0x7fffffff) return LH_ERR_UNSUPPORTED;
+  pool_score_kernel<D, P, L><<<dim3((unsigned)blocks, njobs), kPoolThreads, 0, st>>>(jobs, dm);
+  return check_launch();
+}
+
+template <int D, int P>
+int launch_pool_dp(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+  switch (dm.L) {
+    case 2: return launch_pool_t<D, P, 2>(jobs, njobs, dm, st);
+    case 3: return launch_pool_t<D, P, 3>(jobs, njobs, dm, st);
+    case 4: return launch_pool_t<D, P, 4>(jobs, njobs, dm, st);
+    case 5:
+      if constexpr (P <= 4) return launch_pool_t<D, P, 5>(jobs, njobs, dm, st);
+      return LH_ERR_UNSUPPORTED;
+    default: return LH_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+int launch_pool_d(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+  switch (dm.p) {
+    case 2: return launch_pool_dp<D, 2>(jobs, njobs, dm, st);
+    case 4: return launch_pool_dp<D, 4>(jobs, njobs, dm, st);
+    case 8: return launch_pool_dp<D, 8>(jobs, njobs, dm, st);
+    default: return LH_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+int launch_gather_d(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st) {
+  constexpr int G = D / 8;
+  const int64_t rows = (int64_t)dm.BH * dm.S;
+  const int64_t blocks = (rows + 256 / G - 1) / (256 / G);
+  dim3 grid((unsigned)blocks, njobs);
+  switch (dm.p) {
+    case 2: gather_kernel<D, 2><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
+    case 4: gather_kernel<D, 4><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
+    case 8: gather_kernel<D, 8><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
+    default: return LH_ERR_UNSUPPORTED;
+  }
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_pool_score(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+  if (dm.L < 2) return LH_OK;  // a single level has nothing to pool and nothing to score
+  KernelTimer timer("pool_score", st);
+  return dm.d == 64 ? launch_pool_d<64>(jobs, njobs, dm, st) : launch_pool_d<128>(jobs, njobs, dm, st);
+}
+
+int launch_gather(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st) {
+  KernelTimer timer("gather", st);
+  return dm.d == 64 ? launch_gather_d<64>(jobs, njobs, idx_g, dm, st)
+                    : launch_gather_d<128>(jobs, njobs, idx_g, dm, st);
+}
+
+}  // namespace lh

@@ -1,0 +1,334 @@
+"""Thin Python binding of ``liblh.so`` (the C ABI declared in ``include/lh.h``).
+
+Only argument marshalling happens here: every step of the layer runs in the library's CUDA kernels.  PyTorch
+provides device memory and the current stream.  Function names match the C entry points.  Importing this module
+raises when the library has not been built; there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblh.so")
+
+LH_OK = 0
+LH_ERR_INVALID_ARG = 1
+LH_ERR_UNSUPPORTED = 2
+LH_ERR_CUDA = 3
+LH_ERR_TIMEOUT = 4
+LH_ERR_WORKSPACE = 5
+
+
+class LhParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "L", "p", "k", "C", "flags")]
+
+
+class LhCtxLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in ("qg", "kg", "vg", "og", "lse", "idx_g", "slot", "total")]
+
+
+class LhKernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("ms", ctypes.c_double)]
+
+
+class LighthouseError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {error_string(status)} (status {status})")
+
+
+_P = ctypes.POINTER(LhParams)
+_vp = ctypes.c_void_p
+_SIGS = {
+    "lh_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lh_validate": (ctypes.c_int, [_P]),
+    "lh_S": (ctypes.c_int64, [_P]),
+    "lh_level_size": (ctypes.c_int64, [_P, ctypes.c_int]),
+    "lh_level_offset": (ctypes.c_int64, [_P, ctypes.c_int]),
+    "lh_pyramid_rows": (ctypes.c_int64, [_P]),
+    "lh_score_rows": (ctypes.c_int64, [_P]),
+    "lh_slot_rows": (ctypes.c_int64, [_P]),
+    "lh_ctx_bytes": (ctypes.c_size_t, [_P]),
+    "lh_ctx_layout": (ctypes.c_int, [_P, ctypes.POINTER(LhCtxLayout)]),
+    "lh_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "lh_pool": (ctypes.c_int, [_P, _vp, _vp, _vp]),
+    "lh_score_topk": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "lh_gather": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "lh_attend": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "lh_scatter": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp]),
+    "lh_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "lh_backward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "lh_scatter_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp]),
+    "lh_attend_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "lh_get_status": (ctypes.c_int, [_vp]),
+    "lh_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "lh_profile_read": (ctypes.c_int, [ctypes.POINTER(LhKernelTime), ctypes.c_int]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hierarchical_sparse_attention_avg_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+# ------------------------------------------------------------------------------------------------------------
+# Parameters and host-only queries
+# ------------------------------------------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class Params:
+    B: int
+    H: int
+    N: int
+    d: int
+    L: int
+    p: int
+    k: int
+    C: int
+
+    def c(self) -> LhParams:
+        return LhParams(self.B, self.H, self.N, self.d, self.L, self.p, self.k, self.C, 0)
+
+
+def error_string(status: int) -> str:
+    return _lib.lh_error_string(status).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != LH_OK:
+        raise LighthouseError(rc, where)
+
+
+def lh_validate(P: Params) -> int:
+    return _lib.lh_validate(ctypes.byref(P.c()))
+
+
+def lh_S(P: Params) -> int:
+    return _lib.lh_S(ctypes.byref(P.c()))
+
+
+def lh_level_size(P: Params, level: int) -> int:
+    return _lib.lh_level_size(ctypes.byref(P.c()), level)
+
+
+def lh_level_offset(P: Params, level: int) -> int:
+    return _lib.lh_level_offset(ctypes.byref(P.c()), level)
+
+
+def lh_pyramid_rows(P: Params) -> int:
+    return _lib.lh_pyramid_rows(ctypes.byref(P.c()))
+
+
+def lh_score_rows(P: Params) -> int:
+    return _lib.lh_score_rows(ctypes.byref(P.c()))
+
+
+def lh_slot_rows(P: Params) -> int:
+    return _lib.lh_slot_rows(ctypes.byref(P.c()))
+
+
+def lh_ctx_bytes(P: Params) -> int:
+    return _lib.lh_ctx_bytes(ctypes.byref(P.c()))
+
+
+def lh_workspace_bytes(P: Params) -> int:
+    return _lib.lh_workspace_bytes(ctypes.byref(P.c()))
+
+
+def lh_ctx_layout(P: Params) -> LhCtxLayout:
+    out = LhCtxLayout()
+    _check(_lib.lh_ctx_layout(ctypes.byref(P.c()), ctypes.byref(out)), "lh_ctx_layout")
+    return out
+
+
+# ------------------------------------------------------------------------------------------------------------
+# Device entry points (torch tensors in, torch tensors out)
+# ------------------------------------------------------------------------------------------------------------
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _bf16(t, shape, name):
+    if t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected bf16 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def new_workspace(P: Params, device) -> torch.Tensor:
+    return torch.empty(lh_workspace_bytes(P), dtype=torch.uint8, device=device)
+
+
+def new_ctx(P: Params, device) -> torch.Tensor:
+    return torch.empty(lh_ctx_bytes(P), dtype=torch.uint8, device=device)
+
+
+def ctx_views(P: Params, ctx: torch.Tensor) -> dict:
+    """Typed views of the saved-context buffer written by ``lh_forward``."""
+    lay = lh_ctx_layout(P)
+    S, rows = lh_S(P), P.B * P.H
+
+    def view(off, n, dtype, shape):
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return ctx[off: off + nbytes].view(dtype).view(*shape)
+
+    g = (P.B, P.H, S, P.d)
+    return dict(qg=view(lay.qg, rows * S * P.d, torch.bfloat16, g), kg=view(lay.kg, rows * S * P.d, torch.bfloat16, g),
+                vg=view(lay.vg, rows * S * P.d, torch.bfloat16, g), og=view(lay.og, rows * S * P.d, torch.bfloat16, g),
+                lse=view(lay.lse, rows * S, torch.float32, (P.B, P.H, S)),
+                idx_g=view(lay.idx_g, rows * S, torch.int32, (P.B, P.H, S)),
+                slot=view(lay.slot, rows * lh_slot_rows(P), torch.int32, (P.B, P.H, lh_slot_rows(P))))
+
+
+def lh_pool(P: Params, x, pyr=None):
+    _bf16(x, (P.B, P.H, P.N, P.d), "x")
+    if pyr is None:
+        pyr = torch.empty((P.B, P.H, lh_pyramid_rows(P), P.d), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.lh_pool(ctypes.byref(P.c()), _ptr(x), _ptr(pyr), _stream(x.device)), "lh_pool")
+    return pyr
+
+
+def lh_score_topk(P: Params, k, scores_in=None, scores_out=None, idx_g=None, slot=None, ws=None):
+    dev = k.device
+    _bf16(k, (P.B, P.H, P.N, P.d), "k")
+    if idx_g is None:
+        idx_g = torch.empty((P.B, P.H, lh_S(P)), dtype=torch.int32, device=dev)
+    if slot is None:
+        slot = torch.empty((P.B, P.H, lh_slot_rows(P)), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = new_workspace(P, dev)
+    for t in (scores_in, scores_out):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (P.B, P.H, lh_score_rows(P))):
+            raise ValueError("scores must be fp32 [B, H, lh_score_rows]")
+    rc = _lib.lh_score_topk(ctypes.byref(P.c()), _ptr(k), _ptr(scores_in), _ptr(scores_out), _ptr(idx_g), _ptr(slot),
+                            _ptr(ws), ws.numel(), _stream(dev))
+    _check(rc, "lh_score_topk")
+    return idx_g, slot
+
+
+def lh_gather(P: Params, q, k, v, q_pyr, k_pyr, v_pyr, idx_g, out=None):
+    dev = q.device
+    S = lh_S(P)
+    if out is None:
+        out = tuple(torch.empty((P.B, P.H, S, P.d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    qg, kg, vg = out
+    rc = _lib.lh_gather(ctypes.byref(P.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(q_pyr), _ptr(k_pyr), _ptr(v_pyr),
+                        _ptr(idx_g), _ptr(qg), _ptr(kg), _ptr(vg), _stream(dev))
+    _check(rc, "lh_gather")
+    return qg, kg, vg
+
+
+def lh_attend(P: Params, qg, kg, vg, og=None, lse=None):
+    dev = qg.device
+    S = lh_S(P)
+    for t, n in ((qg, "qg"), (kg, "kg"), (vg, "vg")):
+        _bf16(t, (P.B, P.H, S, P.d), n)
+    if og is None:
+        og = torch.empty_like(qg)
+    if lse is None:
+        lse = torch.empty((P.B, P.H, S), dtype=torch.float32, device=dev)
+    _check(_lib.lh_attend(ctypes.byref(P.c()), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(og), _ptr(lse), _stream(dev)),
+           "lh_attend")
+    return og, lse
+
+
+def lh_scatter(P: Params, og, slot, o=None):
+    dev = og.device
+    if o is None:
+        o = torch.empty((P.B, P.H, P.N, P.d), dtype=torch.bfloat16, device=dev)
+    _check(_lib.lh_scatter(ctypes.byref(P.c()), _ptr(og), _ptr(slot), _ptr(o), _stream(dev)), "lh_scatter")
+    return o
+
+
+def lh_forward(P: Params, q, k, v, o=None, ctx=None, ws=None):
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, (P.B, P.H, P.N, P.d), n)
+    if o is None:
+        o = torch.empty_like(q)
+    if ctx is None:
+        ctx = new_ctx(P, dev)
+    if ws is None:
+        ws = new_workspace(P, dev)
+    rc = _lib.lh_forward(ctypes.byref(P.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ctx), _ptr(ws), ws.numel(),
+                         _stream(dev))
+    _check(rc, "lh_forward")
+    return o, ctx
+
+
+def lh_backward(P: Params, dout, ctx, dq=None, dk=None, dv=None, ws=None):
+    dev = dout.device
+    _bf16(dout, (P.B, P.H, P.N, P.d), "dout")
+    dq = torch.empty_like(dout) if dq is None else dq
+    dk = torch.empty_like(dout) if dk is None else dk
+    dv = torch.empty_like(dout) if dv is None else dv
+    if ws is None:
+        ws = new_workspace(P, dev)
+    rc = _lib.lh_backward(ctypes.byref(P.c()), _ptr(dout), _ptr(ctx), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                          ws.numel(), _stream(dev))
+    _check(rc, "lh_backward")
+    return dq, dk, dv
+
+
+def lh_scatter_bwd(P: Params, dout, idx_g, dog=None):
+    dev = dout.device
+    if dog is None:
+        dog = torch.empty((P.B, P.H, lh_S(P), P.d), dtype=torch.bfloat16, device=dev)
+    _check(_lib.lh_scatter_bwd(ctypes.byref(P.c()), _ptr(dout), _ptr(idx_g), _ptr(dog), _stream(dev)),
+           "lh_scatter_bwd")
+    return dog
+
+
+def lh_attend_bwd(P: Params, qg, kg, vg, og, lse, dog, ws=None):
+    dev = qg.device
+    dqg = torch.empty(qg.shape, dtype=torch.float32, device=dev)
+    dkg = torch.empty_like(qg)
+    dvg = torch.empty_like(qg)
+    if ws is None:
+        ws = new_workspace(P, dev)
+    rc = _lib.lh_attend_bwd(ctypes.byref(P.c()), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(og), _ptr(lse), _ptr(dog),
+                            _ptr(dqg), _ptr(dkg), _ptr(dvg), _ptr(ws), ws.numel(), _stream(dev))
+    _check(rc, "lh_attend_bwd")
+    return dqg, dkg, dvg
+
+
+def lh_get_status(device=None) -> int:
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    return _lib.lh_get_status(_stream(dev))
+
+
+def lh_profile_enable(on: bool = True) -> None:
+    _check(_lib.lh_profile_enable(1 if on else 0), "lh_profile_enable")
+
+
+def lh_profile_read() -> dict:
+    """``{kernel name: (launches, summed device ms)}`` since the last read; clears the record."""
+    buf = (LhKernelTime * 64)()
+    n = _lib.lh_profile_read(buf, 64)
+    if n < 0:
+        raise LighthouseError(-n, "lh_profile_read")
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].ms)) for i in range(n)}

@@ -1,0 +1,198 @@
+/*
+ * lh.h — C ABI of liblh.so, the B200 (sm_100a) Lighthouse selection-and-attend layer.
+ *
+ * The layer (Nous Research's "Lighthouse Attention", as described by the pages cited below) runs, per head:
+ *   1. pool    — symmetric L-level average-pool pyramid over Q, K and V with pool factor p;
+ *   2. score   — parameter-free per-head l2 norm of the pooled keys;
+ *   3. top-K   — chunked (stratified) top-K per level, the coarsest level always kept whole;
+ *   4. gather  — the selected entries as one dense, position-ordered sequence of length S, then causal
+ *                attention over it;
+ *   5. scatter — the outputs written back to token positions with a causality-preserving offset;
+ * and the backward of all five (no gradient through scores or indices).
+ *
+ * Page short names used in the citations:
+ *   [W] wispaper.ai, "Lighthouse Attention：预训练长文本的高速公路，训练提速 21 倍且无损恢复"
+ *   [E] encorp.ai, "Услуги по внедряване на AI задават правилния въпрос за Lighthouse Attention"
+ *   [C] clawdbytes.com, "Lighthouse Attention: the training-time hierarchy that makes quadratic attention …"
+ *   [H] news.hamidun.com, "Nous Research introduced Lighthouse Attention to accelerate LLM training"
+ *
+ * Conventions (every entry point):
+ *   - Tensors are DEVICE pointers owned by the caller, contiguous, row-major, last index fastest, 16-byte aligned.
+ *     bf16 tensors are passed as void* (IEEE bfloat16 bit patterns).
+ *   - Sizes: B batch, H heads, N tokens, d head dim, L levels, p pool factor, k picks per level, C chunks per
+ *     level.  w_l = p^l, N_l = N / w_l.  S = sum_{l<=L-2} min(k, N_l) + N_{L-1}.
+ *   - Global pyramid id of entry (l, j): off_l + j with off_l = sum_{l'<l} N_l' (level 0 = raw tokens first).
+ *   - The library never allocates device memory, never synchronises (except lh_get_status) and never throws.
+ *     Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - Scratch memory is the caller's `ws` of at least lh_workspace_bytes(P) bytes.
+ *   - Return value: LH_OK, or an error code.  Argument errors are detected on the host before any launch.
+ *     A device-side wait that exceeds its bound records LH_ERR_TIMEOUT in a device status word that
+ *     lh_get_status reads; no kernel traps.
+ *   - Supported: d in {64, 128}; p in {2, 4, 8}; 1 <= L <= 5 with p^(L-1) <= 512; k / C <= 512.
+ *     Other valid shapes return LH_ERR_UNSUPPORTED.
+ */
+#ifndef LH_H_
+#define LH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LH_OK 0
+#define LH_ERR_INVALID_ARG 1  /* bad sizes, NULL or misaligned pointer, indivisible shapes */
+#define LH_ERR_UNSUPPORTED 2  /* valid layer, but outside what the kernels are built for */
+#define LH_ERR_CUDA 3         /* a CUDA runtime call or launch failed */
+#define LH_ERR_TIMEOUT 4      /* a device wait hit its bound (reported by lh_get_status) */
+#define LH_ERR_WORKSPACE 5    /* ws_bytes smaller than lh_workspace_bytes */
+
+#define LH_MAX_LEVELS 8
+
+/* Layer sizes.  flags is reserved and must be 0. */
+typedef struct lh_params {
+  int32_t B, H, N, d, L, p, k, C;
+  int32_t flags;
+} lh_params;
+
+/* Byte offsets of the saved-context tensors inside the caller's ctx buffer (see lh_forward). */
+typedef struct lh_ctx_layout_t {
+  uint64_t qg, kg, vg, og; /* bf16 [B,H,S,d]: gathered Q, K, V and the attention output */
+  uint64_t lse;            /* fp32 [B,H,S]: natural-log row log-sum-exp of the attention */
+  uint64_t idx_g;          /* int32 [B,H,S]: global pyramid id of gathered row s */
+  uint64_t slot;           /* int32 [B,H,R], R = sum_l N_l: gathered position of entry off_l + j, or -1 */
+  uint64_t total;          /* bytes needed (= lh_ctx_bytes) */
+} lh_ctx_layout_t;
+
+/* ---- host-only queries (no device work) -------------------------------------------------------------- */
+
+/* Static string for a status code. */
+const char* lh_error_string(int status);
+
+/* LH_OK if P describes a valid layer the kernels support, else LH_ERR_INVALID_ARG / LH_ERR_UNSUPPORTED.
+ * Validity: sizes >= 1, p >= 2, p^(L-1) | N, and C | N_l, C | min(k, N_l) for every level l <= L-2 whose
+ * picks are fewer than its entries ([C] "Four-Stage Pipeline…": equal chunks per level). */
+int lh_validate(const lh_params* P);
+
+/* Gathered length S (see conventions), or -1 if P is invalid. */
+int64_t lh_S(const lh_params* P);
+
+/* N_l, or -1 for an invalid P or level. */
+int64_t lh_level_size(const lh_params* P, int level);
+
+/* off_l (global pyramid id of entry (l, 0)), or -1. */
+int64_t lh_level_offset(const lh_params* P, int level);
+
+/* Rows per head of the pyramid written by lh_pool: sum_{l=1}^{L-1} N_l (level l starts at row
+ * sum_{1<=l'<l} N_l'); -1 if invalid. */
+int64_t lh_pyramid_rows(const lh_params* P);
+
+/* Rows per head of the score array: sum_{l=0}^{L-2} N_l (level l starts at row off_l); -1 if invalid. */
+int64_t lh_score_rows(const lh_params* P);
+
+/* Rows per head of the slot map: sum_{l=0}^{L-1} N_l; -1 if invalid. */
+int64_t lh_slot_rows(const lh_params* P);
+
+/* Bytes of the saved context written by lh_forward and read by lh_backward (0 if invalid). */
+size_t lh_ctx_bytes(const lh_params* P);
+
+/* Fills *out with the ctx layout; LH_OK or an error code. */
+int lh_ctx_layout(const lh_params* P, lh_ctx_layout_t* out);
+
+/* Scratch bytes every device entry point of this header needs at most (0 if invalid). */
+size_t lh_workspace_bytes(const lh_params* P);
+
+/* ---- step-wise API ----------------------------------------------------------------------------------- */
+
+/* Step 1, pool ([W] 核心方法 §1 对称金字塔池化; [E] "Какво точно промени Nous Research в attention пътя?").
+ * x: bf16 [B,H,N,d].  pyr: bf16 [B,H,lh_pyramid_rows,d], levels 1..L-1 stacked (finest first).
+ * Pooled value = bf16_RN(block sum / p^l), the sum taken in fp64 recursively over the p children, left to right
+ * (exact mean rounded once whenever the fp64 sum is exact). */
+int lh_pool(const lh_params* P, const void* x, void* pyr, void* stream);
+
+/* Steps 2-3 and the gathered order ([W] 核心方法 §2 层次化选择器; [C] "Four-Stage Pipeline Wraps Standard
+ * FlashAttention").
+ * k: bf16 [B,H,N,d] raw keys.  Scores: squared l2 norm of the pooled key (raw key at level 0), fp64 sum of
+ * squares (eight left to right per group of eight features, then a pairwise tree over the groups), rounded
+ * to fp32, for levels 0..L-2.
+ * scores_in: optional fp32 [B,H,lh_score_rows]; when non-NULL it replaces the computed scores.
+ * scores_out: optional fp32 [B,H,lh_score_rows]; when non-NULL (and scores_in is NULL) receives the scores.
+ * Selection: C equal chunks per level, each keeping its min(k,N_l)/C entries of largest score (ties: lower
+ * index); coarsest level whole.  Order: ascending end token (j+1)*p^l - 1, equal ends coarser level first.
+ * idx_g: int32 [B,H,S] (out).  slot: int32 [B,H,lh_slot_rows] (out).  ws: scratch. */
+int lh_score_topk(const lh_params* P, const void* k, const float* scores_in, float* scores_out, int32_t* idx_g,
+                  int32_t* slot, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 4a, gather ([W] 核心方法 §3; [E] "Какво точно промени…").  q,k,v: bf16 [B,H,N,d];
+ * q_pyr,k_pyr,v_pyr: bf16 [B,H,lh_pyramid_rows,d] from lh_pool (may be NULL when L == 1); idx_g from
+ * lh_score_topk.  qg,kg,vg: bf16 [B,H,S,d] (out), row s = pooled value of entry idx_g[s] (raw row at level 0). */
+int lh_gather(const lh_params* P, const void* q, const void* k, const void* v, const void* q_pyr,
+              const void* k_pyr, const void* v_pyr, const int32_t* idx_g, void* qg, void* kg, void* vg,
+              void* stream);
+
+/* Step 4b, causal attention over the gathered sequence ([W] 核心方法 §3 标准 FlashAttention 调用;
+ * [H] "How Lighthouse Attention Works").  og = softmax(qg kg^T / sqrt(d) + causal mask) vg, diagonal included.
+ * qg,kg,vg: bf16 [B,H,S,d]; og: bf16 [B,H,S,d] (out); lse: fp32 [B,H,S] (out, natural log).
+ * Runs on the tcgen05 tensor cores (TMA-fed, TMEM accumulators). */
+int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, void* og, float* lse,
+              void* stream);
+
+/* Step 5, offset scatter-back ([W] figure caption "Scatter-back"; [E] "Как four-stage pipeline…": offset that
+ * preserves causality).  O[t] = sum over levels l of og[slot(l, floor((t+1)/p^l) - 1)] over selected entries
+ * (entry (l,j) reaches tokens (j+1)p^l - 1 .. (j+2)p^l - 2); tokens without a selected candidate get 0.
+ * og: bf16 [B,H,S,d]; slot from lh_score_topk; o: bf16 [B,H,N,d] (out, fp32 sum rounded once). */
+int lh_scatter(const lh_params* P, const void* og, const int32_t* slot, void* o, void* stream);
+
+/* ---- fused API --------------------------------------------------------------------------------------- */
+
+/* Whole forward: q,k,v bf16 [B,H,N,d] -> o bf16 [B,H,N,d].  ctx: device buffer of lh_ctx_bytes(P) bytes that
+ * receives the saved context (layout from lh_ctx_layout) and must stay untouched until lh_backward.
+ * Pooled values, scores and the selection are bit-identical to the step-wise API. */
+int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, void* o, void* ctx, void* ws,
+               size_t ws_bytes, void* stream);
+
+/* Whole backward ([E] "Как four-stage pipeline…": gradients reach Q, K, V only through the gathered values;
+ * [W] 深度洞察).  dout: bf16 [B,H,N,d]; ctx from lh_forward; dq,dk,dv: bf16 [B,H,N,d] (out).
+ * dX[t] = sum_l [(l, floor(t/p^l)) selected] dX_g[slot] / p^l. */
+int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq, void* dk, void* dv, void* ws,
+                size_t ws_bytes, void* stream);
+
+/* ---- test-only pieces of the backward ---------------------------------------------------------------- */
+
+/* dog[s] = bf16_RN(sum_{t=E_s}^{min(E_s + w - 1, N - 1)} dout[t]) for the entry idx_g[s] with end E_s and
+ * window w.  dout: bf16 [B,H,N,d]; dog: bf16 [B,H,S,d] (out). */
+int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, void* dog, void* stream);
+
+/* Causal attention backward over S.  Inputs as lh_attend plus og, lse and dog (bf16 [B,H,S,d]).
+ * dqg: fp32 [B,H,S,d] (out); dkg, dvg: bf16 [B,H,S,d] (out).  ws: scratch. */
+int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const void* og,
+                  const float* lse, const void* dog, float* dqg, void* dkg, void* dvg, void* ws, size_t ws_bytes,
+                  void* stream);
+
+/* ---- tracing ----------------------------------------------------------------------------------------- */
+
+/* Device time of the library's own kernels.  While enabled, every kernel the library enqueues is bracketed by two
+ * CUDA events recorded on the stream it is launched on.  lh_profile_read waits for those events, writes up to
+ * max_entries records {kernel name, launches, summed milliseconds} accumulated since the last read (or enable),
+ * clears them and returns the number of records (or -LH_ERR_CUDA).  Events are created lazily and reused. */
+typedef struct lh_kernel_time_t {
+  char name[32];
+  int32_t launches;
+  double ms;
+} lh_kernel_time_t;
+
+int lh_profile_enable(int on);
+int lh_profile_read(lh_kernel_time_t* out, int max_entries);
+
+/* ---- status ------------------------------------------------------------------------------------------ */
+
+/* Synchronises `stream`, returns the first device-side error recorded since the last call (LH_OK if none)
+ * on the current device, and clears it. */
+int lh_get_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LH_H_ */

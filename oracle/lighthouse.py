@@ -260,6 +260,12 @@ def gather(pyr: list[np.ndarray], lev_g: np.ndarray, j_g: np.ndarray) -> np.ndar
 # Step 4b: dense causal attention over the gathered sequence
 # --------------------------------------------------------------------------------------------------------------
 
+def _above_diagonal(S: int) -> np.ndarray:
+    """Boolean ``[S, S]`` mask of the entries ``b > a`` (key after query)."""
+    idx = np.arange(S)
+    return idx[None, :] > idx[:, None]
+
+
 def causal_attention(qg: np.ndarray, kg: np.ndarray, vg: np.ndarray):
     """``softmax(Q K^T / sqrt(d) + causal mask) V`` and the natural-log row LSE, in float64.
 
@@ -267,7 +273,7 @@ def causal_attention(qg: np.ndarray, kg: np.ndarray, vg: np.ndarray):
     [H] "How Lighthouse Attention Works")."""
     S, d = qg.shape
     logits = (qg @ kg.T) / math.sqrt(d)
-    logits[np.triu_indices(S, 1)] = -np.inf
+    np.putmask(logits, _above_diagonal(S), -np.inf)
     mx = logits.max(axis=1, keepdims=True)
     e = np.exp(logits - mx)
     lsum = e.sum(axis=1, keepdims=True)
@@ -282,7 +288,7 @@ def causal_attention_backward(qg, kg, vg, og, lse, dog):
     S, d = qg.shape
     scale = 1.0 / math.sqrt(d)
     logits = (qg @ kg.T) * scale
-    logits[np.triu_indices(S, 1)] = -np.inf
+    np.putmask(logits, _above_diagonal(S), -np.inf)
     prob = np.exp(logits - lse[:, None])
     dvg = prob.T @ dog
     dprob = dog @ vg.T

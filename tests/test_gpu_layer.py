@@ -1,0 +1,213 @@
+"""GPU parity of every step and of the fused forward/backward against the CPU oracle (small shapes that span
+several 128-row tiles, ragged tails, single-level and whole-pyramid cases).
+
+Pass criteria: pyramid, scores, selection (idx_g, slot) and gathered rows bit-exact; floating-point outputs within
+|d| <= 2e-2 + 2e-2 |ref| elementwise.  All calls go through the C ABI (ctypes binding)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_sparse_attention_avg_b200.inputs import make_inputs, make_scores
+from oracle import lighthouse as O
+from tests._parity import assert_close, bits16, f64
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny-d64": (1, 2, 4096, 64, 3, 4, 256, 8),      # the 4K correctness configuration
+    "tiny-d128": (1, 2, 4096, 128, 3, 4, 256, 8),
+    "ragged-S": (1, 2, 2048, 64, 3, 4, 96, 4),       # S = 320
+    "dense-L1": (1, 2, 640, 128, 1, 4, 8, 1),        # one level: plain causal attention, S = N
+    "dense-L1-ragged": (1, 1, 600, 64, 1, 2, 1, 1),
+    "whole-pyramid": (1, 2, 1024, 64, 3, 4, 1024, 4),  # k >= every level: S = 1344
+    "p2-L5": (1, 1, 2048, 64, 5, 2, 64, 2),
+    "p8-L3-B2": (2, 1, 4096, 128, 3, 8, 64, 4),
+}
+
+
+def _lh():
+    from hierarchical_sparse_attention_avg_b200 import lh
+
+    return lh
+
+
+@pytest.fixture(scope="module", params=list(CASES), ids=list(CASES))
+def case(request, cuda_device):
+    lh = _lh()
+    cfg = CASES[request.param]
+    P, Q = lh.Params(*cfg), O.Params(*cfg)
+    q, k, v, dout = make_inputs(Q.B, Q.H, Q.N, Q.d, seed=0, device="cpu")
+    heads = [(b, h) for b in range(Q.B) for h in range(Q.H)]
+    ref = {bh: O.forward_head(f64(q[bh]), f64(k[bh]), f64(v[bh]), Q) for bh in heads}
+    dev = cuda_device
+    return dict(lh=lh, P=P, Q=Q, heads=heads, ref=ref, q=q.to(dev), k=k.to(dev), v=v.to(dev), dout=dout.to(dev),
+                dout_cpu=dout)
+
+
+def _oracle_idx(case):
+    return np.stack([np.stack([case["ref"][(b, h)]["idx_g"] for h in range(case["Q"].H)]) for b in range(case["Q"].B)])
+
+
+def _oracle_slot(case):
+    return np.stack([np.stack([O.slot_map(case["ref"][(b, h)]["slots"]) for h in range(case["Q"].H)])
+                     for b in range(case["Q"].B)])
+
+
+def test_pool_bit_exact(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    if Q.L == 1:
+        pytest.skip("single level: nothing to pool")
+    for name, key in (("q", "pyr_q"), ("k", "pyr_k"), ("v", "pyr_v")):
+        pyr = lh.lh_pool(P, case[name])
+        got = bits16(pyr)
+        for (b, h) in case["heads"]:
+            want = np.concatenate(case["ref"][(b, h)][key][1:])
+            assert np.array_equal(got[b, h], O.bf16_bits(want)), (name, b, h)
+
+
+def test_scores_and_selection_bit_exact(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    dev = case["q"].device
+    scores = torch.empty((Q.B, Q.H, lh.lh_score_rows(P)), dtype=torch.float32, device=dev)
+    idx_g, slot = lh.lh_score_topk(P, case["k"], scores_out=scores)
+    if Q.L > 1:
+        got = scores.cpu().numpy()
+        for (b, h) in case["heads"]:
+            want = np.concatenate(case["ref"][(b, h)]["scores"])
+            assert np.array_equal(got[b, h].view(np.uint32), want.view(np.uint32)), (b, h)
+    assert np.array_equal(idx_g.cpu().numpy(), _oracle_idx(case))
+    assert np.array_equal(slot.cpu().numpy(), _oracle_slot(case))
+
+
+def test_topk_fed_oracle_scores_bit_exact(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    if Q.L == 1:
+        pytest.skip("single level: no scores")
+    dev = case["q"].device
+    for ties in (False, True):
+        sc = make_scores(Q.B, Q.H, lh.lh_score_rows(P), seed=3, ties=ties)
+        idx_g, slot = lh.lh_score_topk(P, case["k"], scores_in=sc.to(dev))
+        for (b, h) in case["heads"]:
+            per = [sc[b, h, Q.level_offset(lev): Q.level_offset(lev) + Q.level_size(lev)].numpy()
+                   for lev in range(Q.L - 1)]
+            sel = O.select(per, Q)
+            lev_g, j_g, slots = O.gathered_order(sel, Q)
+            assert np.array_equal(idx_g[b, h].cpu().numpy(), O.global_ids(lev_g, j_g, Q)), (ties, b, h)
+            assert np.array_equal(slot[b, h].cpu().numpy(), O.slot_map(slots)), (ties, b, h)
+
+
+def test_gather_bit_exact(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    idx_g, _ = lh.lh_score_topk(P, case["k"])
+    pyrs = [lh.lh_pool(P, case[n]) if Q.L > 1 else None for n in ("q", "k", "v")]
+    outs = lh.lh_gather(P, case["q"], case["k"], case["v"], *pyrs, idx_g)
+    for t, key in zip(outs, ("qg", "kg", "vg")):
+        got = bits16(t)
+        for (b, h) in case["heads"]:
+            assert np.array_equal(got[b, h], O.bf16_bits(case["ref"][(b, h)][key])), (key, b, h)
+
+
+def test_attend_matches_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    dev = case["q"].device
+    qg, kg, vg = (torch.from_numpy(np.stack([np.stack([case["ref"][(b, h)][n] for h in range(Q.H)])
+                                             for b in range(Q.B)])).to(torch.bfloat16).to(dev) for n in ("qg", "kg", "vg"))
+    og, lse = lh.lh_attend(P, qg, kg, vg)
+    for (b, h) in case["heads"]:
+        r = case["ref"][(b, h)]
+        assert_close(f64(og[b, h]), r["og"], what=f"og{(b, h)}")
+        assert_close(f64(lse[b, h]), r["lse"], atol=2e-3, rtol=1e-4, what=f"lse{(b, h)}")
+    assert lh.lh_get_status() == 0
+
+
+def test_scatter_matches_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    dev = case["q"].device
+    S = Q.gathered_length()
+    g = torch.Generator().manual_seed(5)
+    og = torch.randn((Q.B, Q.H, S, Q.d), generator=g).to(torch.bfloat16)
+    slot = torch.from_numpy(_oracle_slot(case)).to(torch.int32)
+    o = lh.lh_scatter(P, og.to(dev), slot.to(dev))
+    for (b, h) in case["heads"]:
+        want = O.scatter(f64(og[b, h]), case["ref"][(b, h)]["slots"], Q)
+        assert_close(f64(o[b, h]), want, atol=1e-6, rtol=2 ** -8, what=f"o{(b, h)}")
+
+
+def test_forward_fused_matches_stepwise_and_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    o, ctx = lh.lh_forward(P, case["q"], case["k"], case["v"])
+    views = lh.ctx_views(P, ctx)
+    assert np.array_equal(views["idx_g"].cpu().numpy(), _oracle_idx(case))
+    assert np.array_equal(views["slot"].cpu().numpy(), _oracle_slot(case))
+    for key in ("qg", "kg", "vg"):
+        got = bits16(views[key])
+        for (b, h) in case["heads"]:
+            assert np.array_equal(got[b, h], O.bf16_bits(case["ref"][(b, h)][key])), (key, b, h)
+    for (b, h) in case["heads"]:
+        assert_close(f64(o[b, h]), case["ref"][(b, h)]["out"], what=f"O{(b, h)}")
+    o2, _ = lh.lh_forward(P, case["q"], case["k"], case["v"])
+    assert torch.equal(o, o2), "forward is not deterministic"
+    assert lh.lh_get_status() == 0
+
+
+def test_backward_matches_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    _, ctx = lh.lh_forward(P, case["q"], case["k"], case["v"])
+    dq, dk, dv = lh.lh_backward(P, case["dout"], ctx)
+    for (b, h) in case["heads"]:
+        rq, rk, rv, _ = O.backward_head(f64(case["dout_cpu"][b, h]), case["ref"][(b, h)], Q)
+        assert_close(f64(dq[b, h]), rq, what=f"dQ{(b, h)}")
+        assert_close(f64(dk[b, h]), rk, what=f"dK{(b, h)}")
+        assert_close(f64(dv[b, h]), rv, what=f"dV{(b, h)}")
+    assert lh.lh_get_status() == 0
+
+
+def test_scatter_bwd_matches_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    idx = torch.from_numpy(_oracle_idx(case)).to(torch.int32).to(case["q"].device)
+    dog = lh.lh_scatter_bwd(P, case["dout"], idx)
+    for (b, h) in case["heads"]:
+        r = case["ref"][(b, h)]
+        want = O.scatter_backward(f64(case["dout_cpu"][b, h]), r["lev_g"], r["j_g"], Q)
+        assert_close(f64(dog[b, h]), want, atol=1e-5, rtol=2 ** -8, what=f"dOg{(b, h)}")
+
+
+def test_attend_bwd_matches_oracle(case):
+    lh, P, Q = case["lh"], case["P"], case["Q"]
+    dev = case["q"].device
+    S = Q.gathered_length()
+    qg, kg, vg = (torch.from_numpy(np.stack([np.stack([case["ref"][(b, h)][n] for h in range(Q.H)])
+                                             for b in range(Q.B)])).to(torch.bfloat16).to(dev) for n in ("qg", "kg", "vg"))
+    og, lse = lh.lh_attend(P, qg, kg, vg)
+    g = torch.Generator().manual_seed(6)
+    dog = torch.randn((Q.B, Q.H, S, Q.d), generator=g).to(torch.bfloat16)
+    dqg, dkg, dvg = lh.lh_attend_bwd(P, qg, kg, vg, og, lse, dog.to(dev))
+    for (b, h) in case["heads"]:
+        r = case["ref"][(b, h)]
+        rq, rk, rv = O.causal_attention_backward(r["qg"], r["kg"], r["vg"], r["og"], r["lse"], f64(dog[b, h]))
+        assert_close(f64(dqg[b, h]), rq, what=f"dQg{(b, h)}")
+        assert_close(f64(dkg[b, h]), rk, what=f"dKg{(b, h)}")
+        assert_close(f64(dvg[b, h]), rv, what=f"dVg{(b, h)}")
+    assert lh.lh_get_status() == 0
+
+
+def test_invalid_arguments_are_rejected_before_launch(case):
+    lh, P = case["lh"], case["P"]
+    x = case["q"]
+    bad = lh.Params(P.B, P.H, P.N, P.d, P.L, 1, P.k, P.C)  # pool factor 1 is never valid
+    with pytest.raises(lh.LighthouseError) as e:
+        lh.lh_pool(bad, x)
+    assert e.value.status == lh.LH_ERR_INVALID_ARG
+    import ctypes
+
+    odd = x.view(-1)[1:]  # misaligned by 2 bytes
+    rc = lh.library().lh_scatter(ctypes.byref(P.c()), odd.data_ptr(), odd.data_ptr(), odd.data_ptr(), None)
+    assert rc == lh.LH_ERR_INVALID_ARG
+    ws = torch.empty(16, dtype=torch.uint8, device=x.device)
+    with pytest.raises(lh.LighthouseError) as e:
+        lh.lh_forward(P, case["q"], case["k"], case["v"], ws=ws)
+    assert e.value.status == lh.LH_ERR_WORKSPACE
+    assert lh.lh_get_status() == 0
