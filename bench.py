@@ -63,10 +63,68 @@ def kernel_work(w: dict) -> dict:
         "gather": ("hbm", BH * 3 * (gather_src + S) * row),
         "attn_fwd": ("tensor", 2.0 * S * S * d * BH),
         "scatter": ("hbm", BH * (N * row + S * row + R * 4)),
-        "scatter_bwd": ("hbm", BH * (N * row + 2 * S * row + S * 4 + S * d * 4)),
+        "scatter_bwd": ("hbm", BH * (N * row + S * d * 4)),
+        "bwd_prep": ("hbm", BH * S * (d * 4 * 2 + d * 2 + 4 + d * 4)),
+        "absmax": ("hbm", BH * S * d * 4),
         "attn_bwd": ("tensor", 5.0 * S * S * d * BH),
         "unpool_bwd": ("hbm", BH * (3 * N * row + S * d * 4 + 2 * S * row + R * 4)),
     }, S
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML every 10 ms in a thread while the timed region runs
+    (read-only queries; no setting of the GPU is changed)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device):
+        import threading
+
+        import pynvml
+
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+        self.samples, self.reasons = [], set()
+        self.stop_ev = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS:
+                    if bits & getattr(nv, attr):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self.stop_ev.wait(0.01)
+
+    def start(self):
+        self.thread.start()
+
+    def stop(self) -> dict | None:
+        self.stop_ev.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def make_clock_sampler(device):
+    try:
+        return NvmlClockSampler(device)
+    except Exception:
+        return ClockSampler(device)
 
 
 class ClockSampler:
@@ -222,7 +280,7 @@ def main():
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    clocks = ClockSampler(dev)
+    clocks = make_clock_sampler(dev)
     clocks.start()
     lh.lh_profile_enable(True)
     lh.lh_profile_read()

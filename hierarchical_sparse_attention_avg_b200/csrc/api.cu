@@ -81,7 +81,7 @@ CtxLayout ctx_layout(const LhDims& dm) {
   c.qg = o; o = align_up(o + rows * dm.d * 2);
   c.kg = o; o = align_up(o + rows * dm.d * 2);
   c.vg = o; o = align_up(o + rows * dm.d * 2);
-  c.og = o; o = align_up(o + rows * dm.d * 2);
+  c.og = o; o = align_up(o + rows * dm.d * 4);
   c.lse = o; o = align_up(o + rows * 4);
   c.idx_g = o; o = align_up(o + rows * 4);
   c.slot = o; o = align_up(o + (size_t)dm.BH * dm.R * 4);
@@ -93,7 +93,7 @@ struct WsLayout {
   // forward / selection
   size_t scores, coarse[3], sel, fwd_total;
   // backward
-  size_t dog, dvec, dqacc, dkg, dvg, bwd_total;
+  size_t dog, dog16, dvec, amax, dinv, dqacc, dkg, dvg, bwd_total;
   size_t total;
 };
 WsLayout ws_layout(const LhDims& dm) {
@@ -106,11 +106,14 @@ WsLayout ws_layout(const LhDims& dm) {
   w.fwd_total = o;
   const size_t rows = (size_t)dm.BH * dm.S;
   o = 0;
-  w.dog = o; o = align_up(o + rows * dm.d * 2);
+  w.dog = o; o = align_up(o + rows * dm.d * 4);    // fp32 window sums
+  w.dog16 = o; o = align_up(o + rows * dm.d * 2);  // fp16, scaled per head
   w.dvec = o; o = align_up(o + rows * 4);
+  w.amax = o; o = align_up(o + (size_t)dm.BH * 4);
+  w.dinv = o; o = align_up(o + (size_t)dm.BH * 4);
   w.dqacc = o; o = align_up(o + rows * dm.d * 4);
-  w.dkg = o; o = align_up(o + rows * dm.d * 2);
-  w.dvg = o; o = align_up(o + rows * dm.d * 2);
+  w.dkg = o; o = align_up(o + rows * dm.d * 4);
+  w.dvg = o; o = align_up(o + rows * dm.d * 4);
   w.bwd_total = o;
   w.total = w.fwd_total > w.bwd_total ? w.fwd_total : w.bwd_total;
   if (w.total == 0) w.total = kAlign;
@@ -160,14 +163,14 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-int make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh) {
+int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return LH_ERR_CUDA;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)bh};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
@@ -333,7 +336,7 @@ int lh_gather(const lh_params* P, const void* q, const void* k, const void* v, c
   return launch_gather(jobs, 3, idx_g, dm, (cudaStream_t)stream);
 }
 
-int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, void* og, float* lse,
+int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, float* og, float* lse,
               void* stream) {
   LhDims dm;
   LH_TRY(prepare(P, &dm));
@@ -342,7 +345,7 @@ int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg
   return launch_attn_fwd(qg, kg, vg, og, lse, dm, (cudaStream_t)stream);
 }
 
-int lh_scatter(const lh_params* P, const void* og, const int32_t* slot, void* o, void* stream) {
+int lh_scatter(const lh_params* P, const float* og, const int32_t* slot, void* o, void* stream) {
   LhDims dm;
   LH_TRY(prepare(P, &dm));
   if (!aligned16(og) || !aligned16(slot) || !aligned16(o)) return LH_ERR_INVALID_ARG;
@@ -398,9 +401,10 @@ int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, 
   }
   LH_TRY(launch_gather(gj, 3, idx_g, dm, st));
   // 4b: attention over the gathered sequence
-  LH_TRY(launch_attn_fwd(cb + c.qg, cb + c.kg, cb + c.vg, cb + c.og, reinterpret_cast<float*>(cb + c.lse), dm, st));
+  float* og = reinterpret_cast<float*>(cb + c.og);
+  LH_TRY(launch_attn_fwd(cb + c.qg, cb + c.kg, cb + c.vg, og, reinterpret_cast<float*>(cb + c.lse), dm, st));
   // 5: scatter back
-  return launch_scatter(cb + c.og, slot, o, dm, st);
+  return launch_scatter(og, slot, o, dm, st);
 }
 
 int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq, void* dk, void* dv, void* ws,
@@ -417,23 +421,31 @@ int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq,
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const int32_t* idx_g = reinterpret_cast<const int32_t*>(cb + c.idx_g);
   const int32_t* slot = reinterpret_cast<const int32_t*>(cb + c.slot);
+  float* dog = reinterpret_cast<float*>(wsb + w.dog);
   float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  float* dinv = reinterpret_cast<float*>(wsb + w.dinv);
   float* dqacc = reinterpret_cast<float*>(wsb + w.dqacc);
-  LH_TRY(launch_scatter_bwd(dout, idx_g, wsb + w.dog, cb + c.og, dvec, dqacc, dm, st));
-  LH_TRY(launch_attn_bwd(cb + c.qg, cb + c.kg, cb + c.vg, wsb + w.dog, reinterpret_cast<const float*>(cb + c.lse),
-                         dvec, dqacc, wsb + w.dkg, wsb + w.dvg, dm, st));
-  return launch_unpool_bwd(dqacc, wsb + w.dkg, wsb + w.dvg, slot, dq, dk, dv, dm, st);
+  float* dkg = reinterpret_cast<float*>(wsb + w.dkg);
+  float* dvg = reinterpret_cast<float*>(wsb + w.dvg);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(wsb + w.amax);
+  if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
+  LH_TRY(launch_scatter_bwd(dout, idx_g, dog, amax, dm, st));
+  LH_TRY(launch_bwd_prep(dog, reinterpret_cast<const float*>(cb + c.og), amax, wsb + w.dog16, dvec, dinv, dqacc, dm,
+                         st));
+  LH_TRY(launch_attn_bwd(cb + c.qg, cb + c.kg, cb + c.vg, wsb + w.dog16, reinterpret_cast<const float*>(cb + c.lse),
+                         dvec, dinv, dqacc, dkg, dvg, dm, st));
+  return launch_unpool_bwd(dqacc, dkg, dvg, slot, dq, dk, dv, dm, st);
 }
 
-int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, void* dog, void* stream) {
+int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, float* dog, void* stream) {
   LhDims dm;
   LH_TRY(prepare(P, &dm));
   if (!aligned16(dout) || !aligned16(idx_g) || !aligned16(dog)) return LH_ERR_INVALID_ARG;
-  return launch_scatter_bwd(dout, idx_g, dog, nullptr, nullptr, nullptr, dm, (cudaStream_t)stream);
+  return launch_scatter_bwd(dout, idx_g, dog, nullptr, dm, (cudaStream_t)stream);
 }
 
-int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const void* og,
-                  const float* lse, const void* dog, float* dqg, void* dkg, void* dvg, void* ws, size_t ws_bytes,
+int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const float* og,
+                  const float* lse, const float* dog, float* dqg, float* dkg, float* dvg, void* ws, size_t ws_bytes,
                   void* stream) {
   LhDims dm;
   LH_TRY(prepare(P, &dm));
@@ -443,9 +455,14 @@ int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void
     return LH_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(dm);
   if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
-  float* dvec = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.dvec);
-  LH_TRY(launch_attn_prep(og, dog, dvec, dqg, dm, st));
-  return launch_attn_bwd(qg, kg, vg, dog, lse, dvec, dqg, dkg, dvg, dm, st);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  float* dinv = reinterpret_cast<float*>(wsb + w.dinv);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(wsb + w.amax);
+  if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
+  LH_TRY(launch_absmax(dog, amax, dm, st));
+  LH_TRY(launch_bwd_prep(dog, og, amax, wsb + w.dog16, dvec, dinv, dqg, dm, st));
+  return launch_attn_bwd(qg, kg, vg, wsb + w.dog16, lse, dvec, dinv, dqg, dkg, dvg, dm, st);
 }
 
 int lh_get_status(void* stream) {

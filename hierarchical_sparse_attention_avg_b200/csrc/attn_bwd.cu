@@ -14,6 +14,11 @@
 //   thread (one feature) adds its 128 values to the fp32 dQ accumulator in global memory: a warp's 32 lanes
 //   touch 32 consecutive floats of one row, so every atomic instruction is one coalesced 128-byte reduction.
 // For d = 64 the dQ^T product still uses M = 128; lanes 64..127 are ignored.
+// Operands are fp16 (gathered Q, K, V exactly; P in [0, 1]; dO_g and dS scaled per head by a power of two so
+// that their largest magnitudes sit near 2^10): the layer's window-summed dO_g makes the dS and dV sums cancel
+// strongly, and bf16 operands (8-bit significands) were measured to exceed the 2e-2 + 2e-2|ref| tolerance where
+// fp16 (11-bit) stays within it at the same tensor-core rate.  Results are multiplied by the inverse scale; a
+// dS beyond the fp16 range records LH_ERR_RANGE.
 #include "internal.h"
 
 namespace lh {
@@ -43,8 +48,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const float* __restrict__ lse, const float* __restrict__ dvec, float* __restrict__ dqacc,
-                    __nv_bfloat16* __restrict__ dkg, __nv_bfloat16* __restrict__ dvg, int S, int ntiles,
+                    const float* __restrict__ lse, const float* __restrict__ dvec, const float* __restrict__ dinv,
+                    float* __restrict__ dqacc, float* __restrict__ dkg, float* __restrict__ dvg, int S, int ntiles,
                     float scale, int* status) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -86,9 +91,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tDK = tmem + 256 + D; // dK accumulator (D columns)
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-  constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // both operands K-major
-  constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);   // A K-major, B MN-major
-  constexpr uint32_t idesc_dq = idesc_bf16_f32(128, 128, 1, 1);  // both operands MN-major
+  constexpr uint32_t idesc_kk = idesc_f32acc(kFmtF16, 128, 128, 0, 0);  // both operands K-major
+  constexpr uint32_t idesc_acc = idesc_f32acc(kFmtF16, 128, D, 0, 1);   // A K-major, B MN-major
+  constexpr uint32_t idesc_dq = idesc_f32acc(kFmtF16, 128, 128, 1, 1);  // both operands MN-major
+  const float inv_scale = dinv[bh];                                     // undoes the per-head dO_g scale
 
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(bar_kv, 2 * Lay::TILE);
@@ -122,13 +128,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(sb + Lay::K + koff, 16, 1024), sdesc_sw128(sb + Lay::Q + koff, 16, 1024),
+          umma_ss(tS, sdesc_sw128(sb + Lay::K + koff, 16, 1024), sdesc_sw128(sb + Lay::Q + koff, 16, 1024),
                        idesc_kk, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tDP, sdesc_sw128(sb + Lay::V + koff, 16, 1024), sdesc_sw128(sb + Lay::DO + koff, 16, 1024),
+          umma_ss(tDP, sdesc_sw128(sb + Lay::V + koff, 16, 1024), sdesc_sw128(sb + Lay::DO + koff, 16, 1024),
                        idesc_kk, kk > 0);
         }
         umma_commit(bar_mm1);
@@ -147,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool diag = (i == kt);
     uint8_t* sP = smem + Lay::P;
     uint8_t* sDS = smem + Lay::DS;
+    float ds_max = 0.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float sv[32], dp[32];
@@ -162,18 +169,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pv = ex2(sv[q8 * 8 + e] * scale_log2 - s_lse[qc]);
           if (diag && qc < r) pv = 0.f;        // query qc does not see key r
           p[e] = pv;
-          ds[e] = pv * (dp[q8 * 8 + e] - s_d[qc]) * scale;
+          ds[e] = pv * (dp[q8 * 8 + e] - s_d[qc]) * scale;  // scaled by the head's dO_g scale
+          ds_max = fmaxf(ds_max, fabsf(ds[e]));
         }
         const int col = c * 32 + q8 * 8;
         const uint32_t off = (col >> 6) * 16384 + sw128_offset(r, (col & 63) >> 3);
         *reinterpret_cast<uint4*>(sP + off) =
-            make_uint4(pack_bf16x2_rn(p[0], p[1]), pack_bf16x2_rn(p[2], p[3]), pack_bf16x2_rn(p[4], p[5]),
-                       pack_bf16x2_rn(p[6], p[7]));
+            make_uint4(pack_half2_rn(p[0], p[1]), pack_half2_rn(p[2], p[3]), pack_half2_rn(p[4], p[5]),
+                       pack_half2_rn(p[6], p[7]));
         *reinterpret_cast<uint4*>(sDS + off) =
-            make_uint4(pack_bf16x2_rn(ds[0], ds[1]), pack_bf16x2_rn(ds[2], ds[3]), pack_bf16x2_rn(ds[4], ds[5]),
-                       pack_bf16x2_rn(ds[6], ds[7]));
+            make_uint4(pack_half2_rn(ds[0], ds[1]), pack_half2_rn(ds[2], ds[3]), pack_half2_rn(ds[4], ds[5]),
+                       pack_half2_rn(ds[6], ds[7]));
       }
     }
+    if (__any_sync(0xffffffffu, !(ds_max <= 65504.f)) && lane == 0) set_status(status, LH_ERR_RANGE);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -182,14 +191,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk) {  // reduction over the 128 query rows
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        umma_bf16_ss(tDV, sdesc_sw128(sb + Lay::P + aoff, 16, 1024), sdesc_sw128(sb + Lay::DO + kk * 2048, 16384, 1024),
+        umma_ss(tDV, sdesc_sw128(sb + Lay::P + aoff, 16, 1024), sdesc_sw128(sb + Lay::DO + kk * 2048, 16384, 1024),
                      idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-        umma_bf16_ss(tDK, sdesc_sw128(sb + Lay::DS + aoff, 16, 1024), sdesc_sw128(sb + Lay::Q + kk * 2048, 16384, 1024),
+        umma_ss(tDK, sdesc_sw128(sb + Lay::DS + aoff, 16, 1024), sdesc_sw128(sb + Lay::Q + kk * 2048, 16384, 1024),
                      idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk) {  // reduction over the 128 key rows
-        umma_bf16_ss(tS, sdesc_sw128(sb + Lay::K + kk * 2048, 16384, 1024),
+        umma_ss(tS, sdesc_sw128(sb + Lay::K + kk * 2048, 16384, 1024),
                      sdesc_sw128(sb + Lay::DS + kk * 2048, 16384, 1024), idesc_dq, kk > 0);
       }
       umma_commit(bar_mm2);
@@ -218,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int q = i * kTile + c * 32 + e;
-          if (q < S) atomicAdd(dqacc + ((int64_t)bh * S + q) * D + r, v[e]);
+          if (q < S) atomicAdd(dqacc + ((int64_t)bh * S + q) * D + r, v[e] * inv_scale);
         }
       }
     }
@@ -232,18 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       const uint32_t tacc = which == 0 ? tDV : tDK;
-      __nv_bfloat16* dst_base = which == 0 ? dvg : dkg;
+      float* dst_base = which == 0 ? dvg : dkg;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
         tmem_ld32(tacc + lane_base + c * 32, v);
         tmem_ld_wait();
         if (krow < S) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_base + ((int64_t)bh * S + krow) * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(dst_base + ((int64_t)bh * S + krow) * D + c * 32);
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8)
-            dst[q8] = make_uint4(pack_bf16x2_rn(v[q8 * 8 + 0], v[q8 * 8 + 1]), pack_bf16x2_rn(v[q8 * 8 + 2], v[q8 * 8 + 3]),
-                                 pack_bf16x2_rn(v[q8 * 8 + 4], v[q8 * 8 + 5]), pack_bf16x2_rn(v[q8 * 8 + 6], v[q8 * 8 + 7]));
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
+                                  v[q4 * 4 + 3] * inv_scale);
         }
       }
     }
@@ -262,29 +271,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-int launch_bwd_t(const void* qg, const void* kg, const void* vg, const void* dog, const float* lse, const float* dvec,
-                 float* dqacc, void* dkg, void* dvg, const LhDims& dm, cudaStream_t st) {
+int launch_bwd_t(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse, const float* dvec,
+                 const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
-  if (make_tmap_bf16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_bf16_3d(&mk, kg, D, dm.S, dm.BH) ||
-      make_tmap_bf16_3d(&mv, vg, D, dm.S, dm.BH) || make_tmap_bf16_3d(&mdo, dog, D, dm.S, dm.BH))
+  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH) ||
+      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH))
     return LH_ERR_CUDA;
   const int smem = BwdLayout<D>::BYTES + 1024;
   if (cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LH_ERR_CUDA;
   const int nt = (dm.S + kTile - 1) / kTile;
   KernelTimer timer("attn_bwd", st);
-  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, lse, dvec, dqacc,
-                                                               (__nv_bfloat16*)dkg, (__nv_bfloat16*)dvg, dm.S, nt,
-                                                               1.0f / sqrtf((float)D), dm.status);
+  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, lse, dvec, dinv, dqacc, dkg, dvg,
+                                                               dm.S, nt, 1.0f / sqrtf((float)D), dm.status);
   return check_launch();
 }
 
 }  // namespace
 
-int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog, const float* lse,
-                    const float* dvec, float* dqacc, void* dkg, void* dvg, const LhDims& dm, cudaStream_t st) {
-  return dm.d == 64 ? launch_bwd_t<64>(qg, kg, vg, dog, lse, dvec, dqacc, dkg, dvg, dm, st)
-                    : launch_bwd_t<128>(qg, kg, vg, dog, lse, dvec, dqacc, dkg, dvg, dm, st);
+int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse,
+                    const float* dvec, const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm,
+                    cudaStream_t st) {
+  return dm.d == 64 ? launch_bwd_t<64>(qg, kg, vg, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dm, st)
+                    : launch_bwd_t<128>(qg, kg, vg, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dm, st);
 }
 
 }  // namespace lh

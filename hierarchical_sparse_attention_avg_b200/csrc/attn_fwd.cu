@@ -8,10 +8,12 @@
 //   TMA (128-byte swizzle) brings K_j and V_j into a two-stage ring while the previous tile computes;
 //   one thread issues S = Q K_j^T (tcgen05.mma, M = N = 128, fp32 accumulator in tensor memory);
 //   every thread owns one query row = one TMEM lane: it reads its 128 scores, applies the causal mask on the
-//   diagonal tile, updates the running max (the reference is only moved when the max grows by more than 2^8,
-//   and O in tensor memory is rescaled only then), exponentiates in base 2 and writes P (bf16) into a
-//   swizzled shared-memory tile;
+//   diagonal tile, updates the running max (O in tensor memory is rescaled when any row of the warp grows),
+//   exponentiates in base 2 and writes P (bf16) into a swizzled shared-memory tile.  Keeping the reference at
+//   the running max makes the dominant key's P exactly 1, so O = P V stays consistent with the fp32 P the
+//   backward recomputes (D = rowsum(dO o O) then matches sum_b P dP);
 //   one thread issues O += P V_j (A = P K-major, B = V_j MN-major, fp32 accumulator in tensor memory).
+// O_g is written in fp32: the backward's D and the scatter-back read it at full accumulator precision.
 // Every wait is bounded; a timeout records LH_ERR_TIMEOUT and the block leaves after draining its own copies
 // and MMAs.
 #include "internal.h"
@@ -24,7 +26,6 @@ constexpr int kThreads = 128;
 constexpr int kTile = 128;                 // query rows and key rows per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct FwdLayout {
@@ -40,7 +41,7 @@ struct FwdLayout {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ og,
+                    const __grid_constant__ CUtensorMap tmV, float* __restrict__ og,
                     float* __restrict__ lse, int S, int ntiles, float scale_log2, int* status) {
   using Lay = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -78,8 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tO = tmem + 128;  // columns [128, 128 + D): output accumulator
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+  constexpr uint32_t idesc_qk = idesc_f32acc(kFmtF16, 128, 128, 0, 0);
+  constexpr uint32_t idesc_pv = idesc_f32acc(kFmtF16, 128, D, 0, 1);
 
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(bar_q, Lay::TILE);
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(sb + Lay::Q + koff, 16, 1024), sdesc_sw128(sK + koff, 16, 1024), idesc_qk,
+          umma_ss(tS, sdesc_sw128(sb + Lay::Q + koff, 16, 1024), sdesc_sw128(sK + koff, 16, 1024), idesc_qk,
                        kk > 0);
         }
         umma_commit(bar_s);
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         s[c][i] = x;
         mx = fmaxf(mx, x);
       }
-    const bool grow = mx > m_run + kRescaleThreshold;
+    const bool grow = mx > m_run;
     const float m_new = grow ? mx : m_run;
     const float alpha = ex2(m_run - m_new);  // 1 without growth; 0 on the first tile
     if (j > 0 && __any_sync(0xffffffffu, grow)) {
@@ -177,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs += p[i];
         }
         const int col = c * 32 + q8 * 8;  // first key column of this 16-byte chunk
-        const uint4 v = make_uint4(pack_bf16x2_rn(p[0], p[1]), pack_bf16x2_rn(p[2], p[3]),
-                                   pack_bf16x2_rn(p[4], p[5]), pack_bf16x2_rn(p[6], p[7]));
+        const uint4 v = make_uint4(pack_half2_rn(p[0], p[1]), pack_half2_rn(p[2], p[3]),
+                                   pack_half2_rn(p[4], p[5]), pack_half2_rn(p[6], p[7]));
         *reinterpret_cast<uint4*>(sP + (col >> 6) * 16384 + sw128_offset(row, (col & 63) >> 3)) = v;
       }
     }
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kk = 0; kk < kTile / 16; ++kk) {
         const uint64_t a = sdesc_sw128(sb + Lay::P + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
         const uint64_t b = sdesc_sw128(sV + kk * 2048, 16384, 1024);
-        umma_bf16_ss(tO, a, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_ss(tO, a, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(bar_o);
     }
@@ -213,13 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tO + lane_base + c * 32, o);
       tmem_ld_wait();
       if (grow_idx < S) {
-        uint4* dst = reinterpret_cast<uint4*>(og + ((int64_t)bh * S + grow_idx) * D + c * 32);
+        float4* dst = reinterpret_cast<float4*>(og + ((int64_t)bh * S + grow_idx) * D + c * 32);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          dst[q8] = make_uint4(pack_bf16x2_rn(o[q8 * 8 + 0] * inv_l, o[q8 * 8 + 1] * inv_l),
-                               pack_bf16x2_rn(o[q8 * 8 + 2] * inv_l, o[q8 * 8 + 3] * inv_l),
-                               pack_bf16x2_rn(o[q8 * 8 + 4] * inv_l, o[q8 * 8 + 5] * inv_l),
-                               pack_bf16x2_rn(o[q8 * 8 + 6] * inv_l, o[q8 * 8 + 7] * inv_l));
+        for (int q4 = 0; q4 < 8; ++q4)
+          dst[q4] = make_float4(o[q4 * 4 + 0] * inv_l, o[q4 * 4 + 1] * inv_l, o[q4 * 4 + 2] * inv_l,
+                                o[q4 * 4 + 3] * inv_l);
       }
     }
     if (grow_idx < S) lse[(int64_t)bh * S + grow_idx] = (m_run + __log2f(l_run)) * kLn2;
@@ -241,11 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-int launch_fwd_t(const void* qg, const void* kg, const void* vg, void* og, float* lse, const LhDims& dm,
+int launch_fwd_t(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
                  cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (make_tmap_bf16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_bf16_3d(&mk, kg, D, dm.S, dm.BH) ||
-      make_tmap_bf16_3d(&mv, vg, D, dm.S, dm.BH))
+  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH) ||
+      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH))
     return LH_ERR_CUDA;
   const int smem = FwdLayout<D>::BYTES + 1024;
   if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -253,14 +252,14 @@ int launch_fwd_t(const void* qg, const void* kg, const void* vg, void* og, float
   const int nt = (dm.S + kTile - 1) / kTile;
   const float scale_log2 = kLog2e / sqrtf((float)D);
   KernelTimer timer("attn_fwd", st);
-  attn_fwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, (__nv_bfloat16*)og, lse, dm.S, nt,
+  attn_fwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, nt,
                                                                scale_log2, dm.status);
   return check_launch();
 }
 
 }  // namespace
 
-int launch_attn_fwd(const void* qg, const void* kg, const void* vg, void* og, float* lse, const LhDims& dm,
+int launch_attn_fwd(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
                     cudaStream_t st) {
   return dm.d == 64 ? launch_fwd_t<64>(qg, kg, vg, og, lse, dm, st) : launch_fwd_t<128>(qg, kg, vg, og, lse, dm, st);
 }

@@ -41,20 +41,29 @@ int launch_pool_score(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStr
 int launch_gather(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st);
 int launch_topk(const float* scores, int32_t* sel, int32_t* slot, const LhDims& dm, cudaStream_t st);
 int launch_order(const int32_t* sel, int32_t* idx_g, int32_t* slot, const LhDims& dm, cudaStream_t st);
-int launch_scatter(const void* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st);
-// dog[s] = window sum of dout; when og/dvec/dqacc are non-null also dvec[s] = <dog[s], og[s]> and dqacc[s] = 0.
-int launch_scatter_bwd(const void* dout, const int32_t* idx_g, void* dog, const void* og, float* dvec,
-                       float* dqacc, const LhDims& dm, cudaStream_t st);
-int launch_attn_prep(const void* og, const void* dog, float* dvec, float* dqacc, const LhDims& dm, cudaStream_t st);
-int launch_unpool_bwd(const float* dqg, const void* dkg, const void* dvg, const int32_t* slot, void* dq, void* dk,
+// og (fp32 [BH, S, d]) is the attention output at accumulator precision.
+int launch_scatter(const float* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st);
+// dog[s] = fp32 window sum of dout; with amax non-null also the per-head maximum magnitude (atomicMax on the bit
+// pattern; amax must start at 0).
+int launch_scatter_bwd(const void* dout, const int32_t* idx_g, float* dog, unsigned int* amax, const LhDims& dm,
+                       cudaStream_t st);
+// Per-head maximum magnitude of an fp32 [BH, S, d] tensor (amax must start at 0).
+int launch_absmax(const float* x, unsigned int* amax, const LhDims& dm, cudaStream_t st);
+// dog16 = fp16(dog * scale_bh), dvec = <dog16, og>, dinv[bh] = 1/scale_bh, dqacc = 0.
+int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax, void* dog16, float* dvec, float* dinv,
+                    float* dqacc, const LhDims& dm, cudaStream_t st);
+int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st);
-int launch_attn_fwd(const void* qg, const void* kg, const void* vg, void* og, float* lse, const LhDims& dm,
+int launch_attn_fwd(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
                     cudaStream_t st);
-int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog, const float* lse,
-                    const float* dvec, float* dqacc, void* dkg, void* dvg, const LhDims& dm, cudaStream_t st);
+// qg, kg, vg, dog16: fp16 [BH, S, d] (dog16 scaled per head); dvec scaled alike; dinv: inverse scales.
+// dqacc (fp32, zeroed) accumulates dQ_g; dkg, dvg (fp32) receive dK_g, dV_g.
+int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse,
+                    const float* dvec, const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm,
+                    cudaStream_t st);
 
-// Encode a 3-D bf16 tensor map over [BH][rows][d] with a {64, 128, 1} box and 128-byte swizzle.
-int make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh);
+// Encode a 3-D fp16 tensor map over [BH][rows][d] with a {64, 128, 1} box and 128-byte swizzle.
+int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh);
 
 inline int check_launch() { return cudaGetLastError() == cudaSuccess ? LH_OK : LH_ERR_CUDA; }
 

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -62,6 +63,26 @@ __device__ __forceinline__ void unpack8(const uint4& r, float (&f)[8]) {
     f[2 * i] = __uint_as_float(w[i] << 16);
     f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
+}
+
+// 8 bf16 values -> 8 fp16 values.  Exact for every bf16 value of magnitude in [2^-14, 65504]; smaller ones are
+// rounded to fp16 subnormals, larger ones become infinities and set *overflow.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& r, bool& overflow) {
+  float f[8];
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+    overflow |= fabsf(f[2 * i]) > 65504.f || fabsf(f[2 * i + 1]) > 65504.f;
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
@@ -195,9 +216,10 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation; issued by one thread.
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit inputs (fp16 or bf16, per the instruction descriptor), fp32
+// accumulation; issued by one thread.
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -212,12 +234,19 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                : "memory");
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D (bit layout of the sm_100 UMMA instruction
-// descriptor: D format [4,6), A format [7,10), B format [10,13), A major bit 15, B major bit 16, N>>3 at
-// [17,23), M>>4 at [24,29)).  major: 0 = K-major, 1 = MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+// Instruction descriptor for kind::f16 with fp32 D (bit layout of the sm_100 UMMA instruction descriptor: D format
+// [4,6), A format [7,10), B format [10,13), A major bit 15, B major bit 16, N>>3 at [17,23), M>>4 at [24,29)).
+// fmt: 0 = fp16, 1 = bf16 (A and B always share it).  major: 0 = K-major, 1 = MN-major.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int fmt, int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr int kFmtF16 = 0;
+constexpr int kFmtBF16 = 1;
+
+__device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start address >> 4 at [0,14), leading

@@ -154,7 +154,9 @@ __device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
   return round_pooled(s, 1.0 / (double)ipow(P, lev), val);
 }
 
-// One group per gathered row (b, h, s): copy (level 0), read (pyramid) or recompute (pooled) the row.
+// One group per gathered row (b, h, s): copy (level 0), read (pyramid) or recompute (pooled) the row, and store
+// it as fp16, the operand format of the attention kernels (every bf16 value of magnitude in [2^-14, 65504] is
+// exact in fp16; a larger one records LH_ERR_RANGE).
 template <int D, int P>
 __global__ void __launch_bounds__(256) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
                                                      LhDims dm) {
@@ -180,7 +182,10 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherJobs jobs, const int3
   } else {
     v = pooled_row<D, P>(x + ((int64_t)bh * dm.N + (int64_t)j * dm.wl[lev]) * D + lane * 8, lev);
   }
-  st16(reinterpret_cast<__nv_bfloat16*>(job.out) + row * D + lane * 8, v);
+  bool overflow = false;
+  const uint4 h = bf16x8_to_f16x8(v, overflow);
+  if (overflow) set_status(dm.status, LH_ERR_RANGE);
+  st16(reinterpret_cast<__half*>(job.out) + row * D + lane * 8, h);
 }
 
 template <int D, int P, int L>

@@ -6,10 +6,14 @@
 // the entry j = floor((t+1)/p^l) - 1 when it is selected.
 //
 // The backward has no gradient through the selection ([E] "Как four-stage pipeline…"; [W] 深度洞察):
-//   scatter backward: dO_g[s] = sum of dO over the window E_s .. min(E_s + w - 1, N - 1);
+//   scatter backward: dO_g[s] = sum of dO over the window E_s .. min(E_s + w - 1, N - 1)   (fp32);
 //   unpool backward:  dX[t] = sum_l dX_g[slot(l, floor(t/p^l))] / p^l over selected entries.
+// Between them, the attention backward takes dO_g as fp16 operands.  dO_g is a sum of up to p^(L-1) rows, so
+// it is scaled per head by a power of two (largest magnitude brought into [2^9, 2^10)) before rounding to
+// fp16; D = rowsum(dO_g o O_g) is formed from the same rounded, scaled values, and the attention backward
+// multiplies its results by the inverse scale.
 //
-// Layout: a group of d/8 lanes per row, each lane 8 features (16 bytes); fp32 accumulation, one bf16 rounding.
+// Layout: a group of d/8 lanes per row, each lane 8 features; fp32 accumulation, one rounding at the end.
 #include "internal.h"
 
 namespace lh {
@@ -29,10 +33,44 @@ __device__ __forceinline__ uint4 pack8_rn(const float (&a)[8]) {
                     pack_bf16x2_rn(a[6], a[7]));
 }
 
+// 8 consecutive fp32 values (32 bytes).
+__device__ __forceinline__ void load8f(const float* p, float (&f)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void store8f(float* p, const float (&f)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// Fold a per-row maximum magnitude m (held by the G lanes of a row group) into amax[bh] with few atomics: rows of
+// a warp are consecutive, so the warp spans one head (one atomic) or two (one atomic per row group).  Clamped
+// idle groups repeat the last row and are harmless for a maximum.
+template <int G>
+__device__ __forceinline__ void head_max_atomic(float m, int bh, bool active, int lane, unsigned int* amax) {
+#pragma unroll
+  for (int off = 1; off < G; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const int bh0 = __shfl_sync(0xffffffffu, bh, 0);
+  if (__all_sync(0xffffffffu, bh == bh0)) {
+#pragma unroll
+    for (int off = G; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0 && active) atomicMax(amax + bh, __float_as_uint(m));
+  } else if (lane == 0 && active) {
+    atomicMax(amax + bh, __float_as_uint(m));
+  }
+}
+
+// Power-of-two scale bringing the largest magnitude `amax` into [2^9, 2^10); 1 for an all-zero head.
+__device__ __forceinline__ float head_scale(float amax) {
+  if (!(amax > 0.f) || !isfinite(amax)) return 1.f;
+  int e;
+  frexpf(amax, &e);  // amax = m 2^e, m in [0.5, 1)
+  return ldexpf(1.f, 10 - e);
+}
+
 template <int D>
-__global__ void __launch_bounds__(256) scatter_kernel(const __nv_bfloat16* __restrict__ og,
-                                                      const int32_t* __restrict__ slot, __nv_bfloat16* __restrict__ o,
-                                                      LhDims dm) {
+__global__ void __launch_bounds__(256) scatter_kernel(const float* __restrict__ og, const int32_t* __restrict__ slot,
+                                                      __nv_bfloat16* __restrict__ o, LhDims dm) {
   constexpr int G = D / 8;
   const int lane = threadIdx.x % G;
   const int64_t row = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
@@ -47,21 +85,19 @@ __global__ void __launch_bounds__(256) scatter_kernel(const __nv_bfloat16* __res
     const int s = sl[dm.off[lev] + j];
     if (s < 0) continue;
     float f[8];
-    unpack8(ld16(og + ((int64_t)bh * dm.S + s) * D + lane * 8), f);
+    load8f(og + ((int64_t)bh * dm.S + s) * D + lane * 8, f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] += f[i];
   }
   st_stream16(o + row * D + lane * 8, pack8_rn(acc));
 }
 
-// One group per gathered row.  Optionally also D[s] = <dO_g[s], O_g[s]> (with the rounded dO_g) for the
-// attention backward, and zeroes the fp32 dQ_g accumulator row.
+// One group per gathered row: dog[s] = fp32 window sum of dout.  With amax non-null, also the running per-head
+// maximum magnitude (non-negative fp32 bit patterns order like their values).
 template <int D>
 __global__ void __launch_bounds__(256) scatter_bwd_kernel(const __nv_bfloat16* __restrict__ dout,
-                                                          const int32_t* __restrict__ idx_g,
-                                                          __nv_bfloat16* __restrict__ dog,
-                                                          const __nv_bfloat16* __restrict__ og, float* __restrict__ dvec,
-                                                          float* __restrict__ dqacc, LhDims dm) {
+                                                          const int32_t* __restrict__ idx_g, float* __restrict__ dog,
+                                                          unsigned int* __restrict__ amax, LhDims dm) {
   constexpr int G = D / 8;
   const int lane = threadIdx.x % G;
   const int64_t total = (int64_t)dm.BH * dm.S;
@@ -96,61 +132,78 @@ __global__ void __launch_bounds__(256) scatter_bwd_kernel(const __nv_bfloat16* _
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] += f[i];
   }
-  const uint4 packed = pack8_rn(acc);
-  if (active) st16(dog + row * D + lane * 8, packed);
-  if (dvec) {
-    float rd[8], of[8];
-    unpack8(packed, rd);
-    unpack8(ld16(og + row * D + lane * 8), of);
-    float dot = 0.f;
+  if (active) store8f(dog + row * D + lane * 8, acc);
+  if (amax) {
+    float m = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dot = fmaf(rd[i], of[i], dot);
-#pragma unroll
-    for (int off = 1; off < G; off <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (active && lane == 0) dvec[row] = dot;
-  }
-  if (dqacc && active) {
-    float4* z = reinterpret_cast<float4*>(dqacc + row * D + lane * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(acc[i]));
+    head_max_atomic<G>(m, bh, active, lane, amax);
   }
 }
 
-// D[s] = <dO_g[s], O_g[s]> and a zeroed fp32 dQ_g accumulator, for the stand-alone attention backward.
+// Per-head maximum magnitude of an fp32 [BH, S, d] tensor (for the stand-alone attention backward).
 template <int D>
-__global__ void __launch_bounds__(256) attn_prep_kernel(const __nv_bfloat16* __restrict__ og,
-                                                        const __nv_bfloat16* __restrict__ dog,
-                                                        float* __restrict__ dvec, float* __restrict__ dqacc,
-                                                        LhDims dm) {
+__global__ void __launch_bounds__(256) absmax_kernel(const float* __restrict__ x, unsigned int* __restrict__ amax,
+                                                     LhDims dm) {
   constexpr int G = D / 8;
   const int lane = threadIdx.x % G;
   const int64_t total = (int64_t)dm.BH * dm.S;
   const int64_t row0 = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
   const bool active = row0 < total;
   const int64_t row = active ? row0 : total - 1;
+  float f[8];
+  load8f(x + row * D + lane * 8, f);
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+  head_max_atomic<G>(m, (int)(row / dm.S), active, lane, amax);
+}
+
+// dog16[s] = fp16_RN(dog[s] * scale_bh), D[s] = <dog16[s], og[s]> (scaled domain), dqacc[s] = 0, and the inverse
+// scale of each head.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__ dog, const float* __restrict__ og,
+                                                       const unsigned int* __restrict__ amax, __half* __restrict__ dog16,
+                                                       float* __restrict__ dvec, float* __restrict__ dinv,
+                                                       float* __restrict__ dqacc, LhDims dm) {
+  constexpr int G = D / 8;
+  const int lane = threadIdx.x % G;
+  const int64_t total = (int64_t)dm.BH * dm.S;
+  const int64_t row0 = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
+  const bool active = row0 < total;
+  const int64_t row = active ? row0 : total - 1;
+  const int bh = (int)(row / dm.S);
+  const float sc = head_scale(__uint_as_float(amax[bh]));
   float a[8], b[8];
-  unpack8(ld16(dog + row * D + lane * 8), a);
-  unpack8(ld16(og + row * D + lane * 8), b);
+  load8f(dog + row * D + lane * 8, a);
+  load8f(og + row * D + lane * 8, b);
+  uint32_t h[4];
   float dot = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dot = fmaf(a[i], b[i], dot);
+  for (int i = 0; i < 4; ++i) {
+    __half2 v = __floats2half2_rn(a[2 * i] * sc, a[2 * i + 1] * sc);
+    h[i] = *reinterpret_cast<uint32_t*>(&v);
+    const float2 r = __half22float2(v);
+    dot = fmaf(r.x, b[2 * i], dot);
+    dot = fmaf(r.y, b[2 * i + 1], dot);
+  }
 #pragma unroll
   for (int off = 1; off < G; off <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   if (active) {
+    st16(dog16 + row * D + lane * 8, make_uint4(h[0], h[1], h[2], h[3]));
     if (lane == 0) dvec[row] = dot;
-    float4* z = reinterpret_cast<float4*>(dqacc + row * D + lane * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0 && row % dm.S == 0) dinv[bh] = 1.f / sc;
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    store8f(dqacc + row * D + lane * 8, z);
   }
 }
 
-// blockIdx.y = 0: dQ from the fp32 accumulator; 1: dK; 2: dV (bf16 gathered gradients).
+// blockIdx.y selects the tensor: 0 = dQ, 1 = dK, 2 = dV (fp32 gathered gradients).
 template <int D>
-__global__ void __launch_bounds__(256) unpool_bwd_kernel(const float* __restrict__ dqg,
-                                                         const __nv_bfloat16* __restrict__ dkg,
-                                                         const __nv_bfloat16* __restrict__ dvg,
-                                                         const int32_t* __restrict__ slot, __nv_bfloat16* dq,
-                                                         __nv_bfloat16* dk, __nv_bfloat16* dv, LhDims dm) {
+__global__ void __launch_bounds__(256) unpool_bwd_kernel(const float* __restrict__ dqg, const float* __restrict__ dkg,
+                                                         const float* __restrict__ dvg, const int32_t* __restrict__ slot,
+                                                         __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                                                         LhDims dm) {
   constexpr int G = D / 8;
   const int which = blockIdx.y;
   const int lane = threadIdx.x % G;
@@ -159,20 +212,14 @@ __global__ void __launch_bounds__(256) unpool_bwd_kernel(const float* __restrict
   const int bh = (int)(row / dm.N);
   const int t = (int)(row % dm.N);
   const int32_t* sl = slot + (int64_t)bh * dm.R;
+  const float* src = which == 0 ? dqg : (which == 1 ? dkg : dvg);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int lev = 0; lev < dm.L; ++lev) {
     const int s = sl[dm.off[lev] + t / dm.wl[lev]];
     if (s < 0) continue;
     const float inv_w = 1.0f / (float)dm.wl[lev];  // exact: power-of-two window
-    const int64_t srow = (int64_t)bh * dm.S + s;
     float f[8];
-    if (which == 0) {
-      const float4* p = reinterpret_cast<const float4*>(dqg + srow * D + lane * 8);
-      const float4 a = p[0], b = p[1];
-      f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-    } else {
-      unpack8(ld16((which == 1 ? dkg : dvg) + srow * D + lane * 8), f);
-    }
+    load8f(src + ((int64_t)bh * dm.S + s) * D + lane * 8, f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = fmaf(f[i], inv_w, acc[i]);
   }
@@ -187,56 +234,58 @@ int blocks_for(int64_t rows) {
 
 }  // namespace
 
-int launch_scatter(const void* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st) {
+int launch_scatter(const float* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st) {
   const int64_t rows = (int64_t)dm.BH * dm.N;
   KernelTimer timer("scatter", st);
   if (dm.d == 64)
-    scatter_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>((const __nv_bfloat16*)og, slot, (__nv_bfloat16*)o, dm);
+    scatter_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
   else
-    scatter_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>((const __nv_bfloat16*)og, slot, (__nv_bfloat16*)o,
-                                                                dm);
+    scatter_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
   return check_launch();
 }
 
-int launch_scatter_bwd(const void* dout, const int32_t* idx_g, void* dog, const void* og, float* dvec, float* dqacc,
-                       const LhDims& dm, cudaStream_t st) {
+int launch_scatter_bwd(const void* dout, const int32_t* idx_g, float* dog, unsigned int* amax, const LhDims& dm,
+                       cudaStream_t st) {
   const int64_t rows = (int64_t)dm.BH * dm.S;
   KernelTimer timer("scatter_bwd", st);
   if (dm.d == 64)
-    scatter_bwd_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g,
-                                                                  (__nv_bfloat16*)dog, (const __nv_bfloat16*)og,
-                                                                  dvec, dqacc, dm);
+    scatter_bwd_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
   else
-    scatter_bwd_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g,
-                                                                    (__nv_bfloat16*)dog, (const __nv_bfloat16*)og,
-                                                                    dvec, dqacc, dm);
+    scatter_bwd_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
   return check_launch();
 }
 
-int launch_attn_prep(const void* og, const void* dog, float* dvec, float* dqacc, const LhDims& dm, cudaStream_t st) {
+int launch_absmax(const float* x, unsigned int* amax, const LhDims& dm, cudaStream_t st) {
   const int64_t rows = (int64_t)dm.BH * dm.S;
-  KernelTimer timer("attn_prep", st);
+  KernelTimer timer("absmax", st);
   if (dm.d == 64)
-    attn_prep_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>((const __nv_bfloat16*)og, (const __nv_bfloat16*)dog,
-                                                                dvec, dqacc, dm);
+    absmax_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(x, amax, dm);
   else
-    attn_prep_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>((const __nv_bfloat16*)og,
-                                                                  (const __nv_bfloat16*)dog, dvec, dqacc, dm);
+    absmax_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(x, amax, dm);
   return check_launch();
 }
 
-int launch_unpool_bwd(const float* dqg, const void* dkg, const void* dvg, const int32_t* slot, void* dq, void* dk,
+int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax, void* dog16, float* dvec, float* dinv,
+                    float* dqacc, const LhDims& dm, cudaStream_t st) {
+  const int64_t rows = (int64_t)dm.BH * dm.S;
+  KernelTimer timer("bwd_prep", st);
+  if (dm.d == 64)
+    bwd_prep_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(dog, og, amax, (__half*)dog16, dvec, dinv, dqacc, dm);
+  else
+    bwd_prep_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(dog, og, amax, (__half*)dog16, dvec, dinv, dqacc, dm);
+  return check_launch();
+}
+
+int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st) {
   const int64_t rows = (int64_t)dm.BH * dm.N;
   KernelTimer timer("unpool_bwd", st);
   if (dm.d == 64)
     unpool_bwd_kernel<64><<<dim3(blocks_for<64>(rows), 3), 256, 0, st>>>(
-        dqg, (const __nv_bfloat16*)dkg, (const __nv_bfloat16*)dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
-        (__nv_bfloat16*)dv, dm);
+        dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
   else
     unpool_bwd_kernel<128><<<dim3(blocks_for<128>(rows), 3), 256, 0, st>>>(
-        dqg, (const __nv_bfloat16*)dkg, (const __nv_bfloat16*)dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
-        (__nv_bfloat16*)dv, dm);
+        dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
   return check_launch();
 }
 

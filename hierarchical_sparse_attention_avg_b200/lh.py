@@ -174,9 +174,18 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _valid(P: Params, where: str) -> None:
+    """Raise the library's own status for invalid or unsupported parameters before sizing any buffer."""
+    _check(lh_validate(P), where)
+
+
+def _typed(t, shape, name, dtype=torch.bfloat16):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
 def _bf16(t, shape, name):
-    if t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name}: expected bf16 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+    _typed(t, shape, name, torch.bfloat16)
 
 
 def new_workspace(P: Params, device) -> torch.Tensor:
@@ -197,14 +206,15 @@ def ctx_views(P: Params, ctx: torch.Tensor) -> dict:
         return ctx[off: off + nbytes].view(dtype).view(*shape)
 
     g = (P.B, P.H, S, P.d)
-    return dict(qg=view(lay.qg, rows * S * P.d, torch.bfloat16, g), kg=view(lay.kg, rows * S * P.d, torch.bfloat16, g),
-                vg=view(lay.vg, rows * S * P.d, torch.bfloat16, g), og=view(lay.og, rows * S * P.d, torch.bfloat16, g),
+    return dict(qg=view(lay.qg, rows * S * P.d, torch.float16, g), kg=view(lay.kg, rows * S * P.d, torch.float16, g),
+                vg=view(lay.vg, rows * S * P.d, torch.float16, g), og=view(lay.og, rows * S * P.d, torch.float32, g),
                 lse=view(lay.lse, rows * S, torch.float32, (P.B, P.H, S)),
                 idx_g=view(lay.idx_g, rows * S, torch.int32, (P.B, P.H, S)),
                 slot=view(lay.slot, rows * lh_slot_rows(P), torch.int32, (P.B, P.H, lh_slot_rows(P))))
 
 
 def lh_pool(P: Params, x, pyr=None):
+    _valid(P, "lh_pool")
     _bf16(x, (P.B, P.H, P.N, P.d), "x")
     if pyr is None:
         pyr = torch.empty((P.B, P.H, lh_pyramid_rows(P), P.d), dtype=torch.bfloat16, device=x.device)
@@ -213,6 +223,7 @@ def lh_pool(P: Params, x, pyr=None):
 
 
 def lh_score_topk(P: Params, k, scores_in=None, scores_out=None, idx_g=None, slot=None, ws=None):
+    _valid(P, "lh_score_topk")
     dev = k.device
     _bf16(k, (P.B, P.H, P.N, P.d), "k")
     if idx_g is None:
@@ -231,10 +242,11 @@ def lh_score_topk(P: Params, k, scores_in=None, scores_out=None, idx_g=None, slo
 
 
 def lh_gather(P: Params, q, k, v, q_pyr, k_pyr, v_pyr, idx_g, out=None):
+    _valid(P, "lh_gather")
     dev = q.device
     S = lh_S(P)
     if out is None:
-        out = tuple(torch.empty((P.B, P.H, S, P.d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+        out = tuple(torch.empty((P.B, P.H, S, P.d), dtype=torch.float16, device=dev) for _ in range(3))
     qg, kg, vg = out
     rc = _lib.lh_gather(ctypes.byref(P.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(q_pyr), _ptr(k_pyr), _ptr(v_pyr),
                         _ptr(idx_g), _ptr(qg), _ptr(kg), _ptr(vg), _stream(dev))
@@ -243,12 +255,13 @@ def lh_gather(P: Params, q, k, v, q_pyr, k_pyr, v_pyr, idx_g, out=None):
 
 
 def lh_attend(P: Params, qg, kg, vg, og=None, lse=None):
+    _valid(P, "lh_attend")
     dev = qg.device
     S = lh_S(P)
     for t, n in ((qg, "qg"), (kg, "kg"), (vg, "vg")):
-        _bf16(t, (P.B, P.H, S, P.d), n)
+        _typed(t, (P.B, P.H, S, P.d), n, torch.float16)
     if og is None:
-        og = torch.empty_like(qg)
+        og = torch.empty(qg.shape, dtype=torch.float32, device=dev)
     if lse is None:
         lse = torch.empty((P.B, P.H, S), dtype=torch.float32, device=dev)
     _check(_lib.lh_attend(ctypes.byref(P.c()), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(og), _ptr(lse), _stream(dev)),
@@ -257,6 +270,7 @@ def lh_attend(P: Params, qg, kg, vg, og=None, lse=None):
 
 
 def lh_scatter(P: Params, og, slot, o=None):
+    _valid(P, "lh_scatter")
     dev = og.device
     if o is None:
         o = torch.empty((P.B, P.H, P.N, P.d), dtype=torch.bfloat16, device=dev)
@@ -265,6 +279,7 @@ def lh_scatter(P: Params, og, slot, o=None):
 
 
 def lh_forward(P: Params, q, k, v, o=None, ctx=None, ws=None):
+    _valid(P, "lh_forward")
     dev = q.device
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _bf16(t, (P.B, P.H, P.N, P.d), n)
@@ -281,6 +296,7 @@ def lh_forward(P: Params, q, k, v, o=None, ctx=None, ws=None):
 
 
 def lh_backward(P: Params, dout, ctx, dq=None, dk=None, dv=None, ws=None):
+    _valid(P, "lh_backward")
     dev = dout.device
     _bf16(dout, (P.B, P.H, P.N, P.d), "dout")
     dq = torch.empty_like(dout) if dq is None else dq
@@ -295,19 +311,26 @@ def lh_backward(P: Params, dout, ctx, dq=None, dk=None, dv=None, ws=None):
 
 
 def lh_scatter_bwd(P: Params, dout, idx_g, dog=None):
+    _valid(P, "lh_scatter_bwd")
     dev = dout.device
     if dog is None:
-        dog = torch.empty((P.B, P.H, lh_S(P), P.d), dtype=torch.bfloat16, device=dev)
+        dog = torch.empty((P.B, P.H, lh_S(P), P.d), dtype=torch.float32, device=dev)
     _check(_lib.lh_scatter_bwd(ctypes.byref(P.c()), _ptr(dout), _ptr(idx_g), _ptr(dog), _stream(dev)),
            "lh_scatter_bwd")
     return dog
 
 
 def lh_attend_bwd(P: Params, qg, kg, vg, og, lse, dog, ws=None):
+    _valid(P, "lh_attend_bwd")
     dev = qg.device
+    S = lh_S(P)
+    for t, n in ((qg, "qg"), (kg, "kg"), (vg, "vg")):
+        _typed(t, (P.B, P.H, S, P.d), n, torch.float16)
+    for t, n in ((og, "og"), (dog, "dog")):
+        _typed(t, (P.B, P.H, S, P.d), n, torch.float32)
     dqg = torch.empty(qg.shape, dtype=torch.float32, device=dev)
-    dkg = torch.empty_like(qg)
-    dvg = torch.empty_like(qg)
+    dkg = torch.empty(qg.shape, dtype=torch.float32, device=dev)
+    dvg = torch.empty(qg.shape, dtype=torch.float32, device=dev)
     if ws is None:
         ws = new_workspace(P, dev)
     rc = _lib.lh_attend_bwd(ctypes.byref(P.c()), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(og), _ptr(lse), _ptr(dog),

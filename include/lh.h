@@ -47,6 +47,7 @@ extern "C" {
 #define LH_ERR_CUDA 3         /* a CUDA runtime call or launch failed */
 #define LH_ERR_TIMEOUT 4      /* a device wait hit its bound (reported by lh_get_status) */
 #define LH_ERR_WORKSPACE 5    /* ws_bytes smaller than lh_workspace_bytes */
+#define LH_ERR_RANGE 6        /* a value left the fp16 range of the attention operands (reported by lh_get_status) */
 
 #define LH_MAX_LEVELS 8
 
@@ -58,7 +59,8 @@ typedef struct lh_params {
 
 /* Byte offsets of the saved-context tensors inside the caller's ctx buffer (see lh_forward). */
 typedef struct lh_ctx_layout_t {
-  uint64_t qg, kg, vg, og; /* bf16 [B,H,S,d]: gathered Q, K, V and the attention output */
+  uint64_t qg, kg, vg;     /* fp16 [B,H,S,d]: gathered Q, K, V (see lh_gather) */
+  uint64_t og;             /* fp32 [B,H,S,d]: attention output over the gathered sequence */
   uint64_t lse;            /* fp32 [B,H,S]: natural-log row log-sum-exp of the attention */
   uint64_t idx_g;          /* int32 [B,H,S]: global pyramid id of gathered row s */
   uint64_t slot;           /* int32 [B,H,R], R = sum_l N_l: gathered position of entry off_l + j, or -1 */
@@ -126,23 +128,26 @@ int lh_score_topk(const lh_params* P, const void* k, const float* scores_in, flo
 
 /* Step 4a, gather ([W] 核心方法 §3; [E] "Какво точно промени…").  q,k,v: bf16 [B,H,N,d];
  * q_pyr,k_pyr,v_pyr: bf16 [B,H,lh_pyramid_rows,d] from lh_pool (may be NULL when L == 1); idx_g from
- * lh_score_topk.  qg,kg,vg: bf16 [B,H,S,d] (out), row s = pooled value of entry idx_g[s] (raw row at level 0). */
+ * lh_score_topk.  qg,kg,vg: fp16 [B,H,S,d] (out), row s = the bf16 pooled value of entry idx_g[s] (raw row at
+ * level 0) converted to fp16, the attention's operand format: exact for magnitudes in [2^-14, 65504]; a larger
+ * value records LH_ERR_RANGE in the device status word. */
 int lh_gather(const lh_params* P, const void* q, const void* k, const void* v, const void* q_pyr,
               const void* k_pyr, const void* v_pyr, const int32_t* idx_g, void* qg, void* kg, void* vg,
               void* stream);
 
 /* Step 4b, causal attention over the gathered sequence ([W] 核心方法 §3 标准 FlashAttention 调用;
  * [H] "How Lighthouse Attention Works").  og = softmax(qg kg^T / sqrt(d) + causal mask) vg, diagonal included.
- * qg,kg,vg: bf16 [B,H,S,d]; og: bf16 [B,H,S,d] (out); lse: fp32 [B,H,S] (out, natural log).
- * Runs on the tcgen05 tensor cores (TMA-fed, TMEM accumulators). */
-int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, void* og, float* lse,
+ * qg,kg,vg: fp16 [B,H,S,d] (as written by lh_gather); og: fp32 [B,H,S,d] (out, accumulator precision); lse: fp32
+ * [B,H,S] (out, natural log).  Runs on the tcgen05 tensor cores (TMA-fed, TMEM accumulators); P enters the PV
+ * product in fp16. */
+int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg, float* og, float* lse,
               void* stream);
 
 /* Step 5, offset scatter-back ([W] figure caption "Scatter-back"; [E] "Как four-stage pipeline…": offset that
  * preserves causality).  O[t] = sum over levels l of og[slot(l, floor((t+1)/p^l) - 1)] over selected entries
  * (entry (l,j) reaches tokens (j+1)p^l - 1 .. (j+2)p^l - 2); tokens without a selected candidate get 0.
- * og: bf16 [B,H,S,d]; slot from lh_score_topk; o: bf16 [B,H,N,d] (out, fp32 sum rounded once). */
-int lh_scatter(const lh_params* P, const void* og, const int32_t* slot, void* o, void* stream);
+ * og: fp32 [B,H,S,d]; slot from lh_score_topk; o: bf16 [B,H,N,d] (out, fp32 sum rounded once). */
+int lh_scatter(const lh_params* P, const float* og, const int32_t* slot, void* o, void* stream);
 
 /* ---- fused API --------------------------------------------------------------------------------------- */
 
@@ -160,14 +165,16 @@ int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq,
 
 /* ---- test-only pieces of the backward ---------------------------------------------------------------- */
 
-/* dog[s] = bf16_RN(sum_{t=E_s}^{min(E_s + w - 1, N - 1)} dout[t]) for the entry idx_g[s] with end E_s and
- * window w.  dout: bf16 [B,H,N,d]; dog: bf16 [B,H,S,d] (out). */
-int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, void* dog, void* stream);
+/* dog[s] = sum_{t=E_s}^{min(E_s + w - 1, N - 1)} dout[t] (fp32 sum) for the entry idx_g[s] with end E_s and
+ * window w.  dout: bf16 [B,H,N,d]; dog: fp32 [B,H,S,d] (out). */
+int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, float* dog, void* stream);
 
-/* Causal attention backward over S.  Inputs as lh_attend plus og, lse and dog (bf16 [B,H,S,d]).
- * dqg: fp32 [B,H,S,d] (out); dkg, dvg: bf16 [B,H,S,d] (out).  ws: scratch. */
-int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const void* og,
-                  const float* lse, const void* dog, float* dqg, void* dkg, void* dvg, void* ws, size_t ws_bytes,
+/* Causal attention backward over S.  qg,kg,vg: fp16 [B,H,S,d]; og: fp32 [B,H,S,d] and lse from lh_attend;
+ * dog: fp32 [B,H,S,d] (gradient of og).  dqg, dkg, dvg: fp32 [B,H,S,d] (out).  ws: scratch.
+ * The tensor-core operands are fp16; dog is scaled per head by a power of two before rounding (its largest
+ * magnitude in [2^9, 2^10)) and the results are scaled back. */
+int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void* vg, const float* og,
+                  const float* lse, const float* dog, float* dqg, float* dkg, float* dvg, void* ws, size_t ws_bytes,
                   void* stream);
 
 /* ---- tracing ----------------------------------------------------------------------------------------- */

@@ -10,6 +10,7 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
+    config.addinivalue_line("markers", "full: full-size benchmark configuration (minutes of CPU oracle time)")
 
 
 @pytest.fixture(scope="session")

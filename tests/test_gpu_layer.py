@@ -99,22 +99,35 @@ def test_topk_fed_oracle_scores_bit_exact(case):
             assert np.array_equal(slot[b, h].cpu().numpy(), O.slot_map(slots)), (ties, b, h)
 
 
-def test_gather_bit_exact(case):
+def _fp16(a):
+    """IEEE round-to-nearest-even to fp16 (exact for the bf16 values of magnitude in [2^-14, 65504])."""
+    return np.asarray(a, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def _oracle_gathered(case, key, dev):
+    """The oracle's gathered rows as the fp16 operands the attention takes."""
+    Q = case["Q"]
+    a = np.stack([np.stack([case["ref"][(b, h)][key] for h in range(Q.H)]) for b in range(Q.B)])
+    return torch.from_numpy(a).to(torch.float16).to(dev)
+
+
+def test_gather_exact(case):
     lh, P, Q = case["lh"], case["P"], case["Q"]
     idx_g, _ = lh.lh_score_topk(P, case["k"])
     pyrs = [lh.lh_pool(P, case[n]) if Q.L > 1 else None for n in ("q", "k", "v")]
     outs = lh.lh_gather(P, case["q"], case["k"], case["v"], *pyrs, idx_g)
     for t, key in zip(outs, ("qg", "kg", "vg")):
-        got = bits16(t)
+        assert t.dtype == torch.float16
+        got = f64(t)
         for (b, h) in case["heads"]:
-            assert np.array_equal(got[b, h], O.bf16_bits(case["ref"][(b, h)][key])), (key, b, h)
+            assert np.array_equal(got[b, h], _fp16(case["ref"][(b, h)][key])), (key, b, h)
+    assert lh.lh_get_status() == 0
 
 
 def test_attend_matches_oracle(case):
     lh, P, Q = case["lh"], case["P"], case["Q"]
     dev = case["q"].device
-    qg, kg, vg = (torch.from_numpy(np.stack([np.stack([case["ref"][(b, h)][n] for h in range(Q.H)])
-                                             for b in range(Q.B)])).to(torch.bfloat16).to(dev) for n in ("qg", "kg", "vg"))
+    qg, kg, vg = (_oracle_gathered(case, n, dev) for n in ("qg", "kg", "vg"))
     og, lse = lh.lh_attend(P, qg, kg, vg)
     for (b, h) in case["heads"]:
         r = case["ref"][(b, h)]
@@ -128,7 +141,7 @@ def test_scatter_matches_oracle(case):
     dev = case["q"].device
     S = Q.gathered_length()
     g = torch.Generator().manual_seed(5)
-    og = torch.randn((Q.B, Q.H, S, Q.d), generator=g).to(torch.bfloat16)
+    og = torch.randn((Q.B, Q.H, S, Q.d), generator=g)
     slot = torch.from_numpy(_oracle_slot(case)).to(torch.int32)
     o = lh.lh_scatter(P, og.to(dev), slot.to(dev))
     for (b, h) in case["heads"]:
@@ -143,9 +156,9 @@ def test_forward_fused_matches_stepwise_and_oracle(case):
     assert np.array_equal(views["idx_g"].cpu().numpy(), _oracle_idx(case))
     assert np.array_equal(views["slot"].cpu().numpy(), _oracle_slot(case))
     for key in ("qg", "kg", "vg"):
-        got = bits16(views[key])
+        got = f64(views[key])
         for (b, h) in case["heads"]:
-            assert np.array_equal(got[b, h], O.bf16_bits(case["ref"][(b, h)][key])), (key, b, h)
+            assert np.array_equal(got[b, h], _fp16(case["ref"][(b, h)][key])), (key, b, h)
     for (b, h) in case["heads"]:
         assert_close(f64(o[b, h]), case["ref"][(b, h)]["out"], what=f"O{(b, h)}")
     o2, _ = lh.lh_forward(P, case["q"], case["k"], case["v"])
@@ -172,18 +185,22 @@ def test_scatter_bwd_matches_oracle(case):
     for (b, h) in case["heads"]:
         r = case["ref"][(b, h)]
         want = O.scatter_backward(f64(case["dout_cpu"][b, h]), r["lev_g"], r["j_g"], Q)
-        assert_close(f64(dog[b, h]), want, atol=1e-5, rtol=2 ** -8, what=f"dOg{(b, h)}")
+        assert_close(f64(dog[b, h]), want, atol=1e-4, rtol=1e-5, what=f"dOg{(b, h)}")
 
 
 def test_attend_bwd_matches_oracle(case):
     lh, P, Q = case["lh"], case["P"], case["Q"]
     dev = case["q"].device
     S = Q.gathered_length()
-    qg, kg, vg = (torch.from_numpy(np.stack([np.stack([case["ref"][(b, h)][n] for h in range(Q.H)])
-                                             for b in range(Q.B)])).to(torch.bfloat16).to(dev) for n in ("qg", "kg", "vg"))
+    qg, kg, vg = (_oracle_gathered(case, n, dev) for n in ("qg", "kg", "vg"))
     og, lse = lh.lh_attend(P, qg, kg, vg)
+    # the gradient of the gathered output as the layer produces it: window sums of a random upstream gradient
     g = torch.Generator().manual_seed(6)
-    dog = torch.randn((Q.B, Q.H, S, Q.d), generator=g).to(torch.bfloat16)
+    dout = torch.randn((Q.N, Q.d), generator=g).to(torch.bfloat16)
+    dog = torch.empty((Q.B, Q.H, S, Q.d), dtype=torch.float32)
+    for (b, h) in case["heads"]:
+        r = case["ref"][(b, h)]
+        dog[b, h] = torch.from_numpy(O.scatter_backward(f64(dout), r["lev_g"], r["j_g"], Q))
     dqg, dkg, dvg = lh.lh_attend_bwd(P, qg, kg, vg, og, lse, dog.to(dev))
     for (b, h) in case["heads"]:
         r = case["ref"][(b, h)]
