@@ -196,6 +196,7 @@ const char* lh_error_string(int status) {
     case LH_ERR_CUDA: return "CUDA error";
     case LH_ERR_TIMEOUT: return "device wait timed out";
     case LH_ERR_WORKSPACE: return "workspace too small";
+    case LH_ERR_RANGE: return "value outside the fp16 operand range";
     default: return "unknown status";
   }
 }

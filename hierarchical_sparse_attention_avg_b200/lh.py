@@ -21,6 +21,7 @@ LH_ERR_UNSUPPORTED = 2
 LH_ERR_CUDA = 3
 LH_ERR_TIMEOUT = 4
 LH_ERR_WORKSPACE = 5
+LH_ERR_RANGE = 6
 
 
 class LhParams(ctypes.Structure):

@@ -100,6 +100,6 @@ def test_k_at_least_level_size_needs_no_divisibility(lh):
 
 
 def test_error_strings(lh):
-    for code in range(6):
+    for code in range(7):
         assert lh.error_string(code)
     assert lh.error_string(99) == "unknown status"
