@@ -29,6 +29,8 @@ WORKLOADS = {
     "ctx98K": dict(B=1, H=16, N=98304, d=64, L=4, p=4, k=2048, C=16),
     "long512K": dict(B=1, H=16, N=524288, d=128, L=4, p=4, k=4096, C=32),
     "stress1M": dict(B=1, H=8, N=1048576, d=128, L=4, p=4, k=4096, C=32),
+    # a smaller d=128 case with the long-context level structure, for profiler captures that must stay small
+    "probe128K": dict(B=1, H=4, N=131072, d=128, L=4, p=4, k=4096, C=32),
 }
 DEFAULT_WORKLOAD = "long512K"
 METRIC = "Lighthouse fwd+bwd tokens/s at N=512K; HBM GB/s and attention TFLOP/s vs peak"
