@@ -478,3 +478,70 @@ int lh_get_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------------------
+// Selection without caller-provided scratch (lh_score_topk_static).
+//
+// Some callers cannot allocate device memory at the point where they need the selection: a runtime that plans
+// all of its device memory once at start-up and forbids allocation on its step path, or a hook inside another
+// framework that is handed only the tensors it reads and writes.  For them this entry point keeps its scratch
+// (the per-level selection lists and, when the caller passes no score buffer, the scores) in one fixed device
+// array owned by the library.
+// ------------------------------------------------------------------------------------------------------------
+
+namespace lh {
+namespace {
+
+// Loaded with the library on every device that uses it and held until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[LH_STATIC_SCRATCH_BYTES];
+
+// Device address of g_static_scratch on the current device, looked up once per device.  The symbol's name is a
+// host-side stand-in in host code, so kernels must be given this address instead.
+int static_scratch_ptr(unsigned char** out) {
+  static std::mutex mu;
+  static unsigned char* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LH_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return LH_ERR_CUDA;
+    cache[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = cache[dev];
+  return LH_OK;
+}
+
+}  // namespace
+}  // namespace lh
+
+extern "C" int lh_score_topk_static(const lh_params* P, const void* k, const float* scores_in, float* scores_out,
+                                    int32_t* idx_g, int32_t* slot, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(idx_g) || !aligned16(slot)) return LH_ERR_INVALID_ARG;
+  const bool own_scores = dm.L >= 2 && !scores_in && !scores_out;
+  if (dm.L >= 2 && !scores_in && !aligned16(k)) return LH_ERR_INVALID_ARG;
+  if (dm.L >= 2 && scores_in && !aligned16(scores_in)) return LH_ERR_INVALID_ARG;
+  if (scores_out && !aligned16(scores_out)) return LH_ERR_INVALID_ARG;
+  // scratch: the selection lists, then (only when the caller gives no score buffer) the scores
+  const size_t sel_bytes = align_up((size_t)dm.BH * dm.Ksel * 4);
+  const size_t need = sel_bytes + (own_scores ? align_up((size_t)dm.BH * dm.Rs * 4) : 0);
+  if (need > (size_t)LH_STATIC_SCRATCH_BYTES) return LH_ERR_WORKSPACE;
+  unsigned char* scratch = nullptr;
+  LH_TRY(static_scratch_ptr(&scratch));
+  int32_t* sel = reinterpret_cast<int32_t*>(scratch);
+  const float* scores = scores_in;
+  if (dm.L >= 2 && !scores_in) {
+    float* dst = scores_out ? scores_out : reinterpret_cast<float*>(scratch + sel_bytes);
+    PoolJobs jobs;
+    memset(&jobs, 0, sizeof(jobs));
+    jobs.job[0].x = k;
+    jobs.job[0].scores = dst;
+    LH_TRY(launch_pool_score(jobs, 1, dm, st));
+    scores = dst;
+  }
+  LH_TRY(launch_topk(scores, sel, slot, dm, st));
+  return launch_order(sel, idx_g, slot, dm, st);
+}

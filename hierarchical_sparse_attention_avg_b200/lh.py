@@ -66,6 +66,7 @@ _SIGS = {
     "lh_scatter_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp]),
     "lh_attend_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "lh_get_status": (ctypes.c_int, [_vp]),
+    "lh_score_topk_static": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
     "lh_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "lh_profile_read": (ctypes.c_int, [ctypes.POINTER(LhKernelTime), ctypes.c_int]),
 }
@@ -356,3 +357,23 @@ def lh_profile_read() -> dict:
     if n < 0:
         raise LighthouseError(-n, "lh_profile_read")
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].ms)) for i in range(n)}
+
+
+LH_STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def lh_score_topk_static(P: Params, k, scores_in=None, scores_out=None, idx_g=None, slot=None):
+    """``lh_score_topk`` without a caller workspace: the library's fixed device scratch array is used instead
+    (for callers that cannot allocate device memory where they select).  Output buffers are created here only
+    for convenience when not given; the library call itself allocates nothing."""
+    _valid(P, "lh_score_topk_static")
+    dev = k.device
+    _bf16(k, (P.B, P.H, P.N, P.d), "k")
+    if idx_g is None:
+        idx_g = torch.empty((P.B, P.H, lh_S(P)), dtype=torch.int32, device=dev)
+    if slot is None:
+        slot = torch.empty((P.B, P.H, lh_slot_rows(P)), dtype=torch.int32, device=dev)
+    rc = _lib.lh_score_topk_static(ctypes.byref(P.c()), _ptr(k), _ptr(scores_in), _ptr(scores_out), _ptr(idx_g),
+                                   _ptr(slot), _stream(dev))
+    _check(rc, "lh_score_topk_static")
+    return idx_g, slot

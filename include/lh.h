@@ -192,6 +192,30 @@ typedef struct lh_kernel_time_t {
 int lh_profile_enable(int on);
 int lh_profile_read(lh_kernel_time_t* out, int max_entries);
 
+/* ---- selection without caller scratch ---------------------------------------------------------------- */
+
+/* Size of the library's fixed device scratch array used by lh_score_topk_static (per device, held from the
+ * first use of the library on that device until the process exits). */
+#define LH_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* The pages have no counterpart to this entry point; it exists for callers that cannot allocate device memory
+ * where they need the selection (for example a runtime that plans all device memory once at start-up and
+ * forbids allocation on its step path, or a hook handed only the tensors it reads and writes).
+ *
+ * Same result as lh_score_topk (same arguments, same kernels, bit-identical idx_g, slot and scores), but the
+ * scratch comes from a fixed device array inside the library instead of a caller workspace, and no device
+ * memory is allocated or freed.  The scratch holds the selection lists (B*H*sum over partially selected levels
+ * of k int32) and, only when both scores_in and scores_out are NULL, the scores (B*H*lh_score_rows fp32), each
+ * rounded up to 256 bytes; a call that needs more than LH_STATIC_SCRATCH_BYTES returns LH_ERR_WORKSPACE before
+ * any launch.  Nothing in the array has to start at zero: every call writes what it later reads.
+ *
+ * The first call on a device looks up the array's device address with cudaGetSymbolAddress (with that device
+ * current) and caches it; make that first call before any stream capture.  All calls on a device share the one
+ * array, which keeps the last call's contents: calls whose work can overlap on the GPU (different streams,
+ * concurrent host threads) race on it and must be serialised by the caller. */
+int lh_score_topk_static(const lh_params* P, const void* k, const float* scores_in, float* scores_out,
+                         int32_t* idx_g, int32_t* slot, void* stream);
+
 /* ---- status ------------------------------------------------------------------------------------------ */
 
 /* Synchronises `stream`, returns the first device-side error recorded since the last call (LH_OK if none)
