@@ -38,6 +38,8 @@ int make_dims(const lh_params* P, LhDims* dm) {
     const int64_t n = P->N / wl;
     dm->Nl[l] = (int)n;
     dm->wl[l] = (int)wl;
+    dm->wlog[l] = 0;
+    while ((int64_t(1) << dm->wlog[l]) < wl) ++dm->wlog[l];  // exact log2 when p is a power of two
     dm->off[l] = (int)R;
     if (l >= 1) dm->poff[l] = (int)Rp;
     int64_t kl = n;

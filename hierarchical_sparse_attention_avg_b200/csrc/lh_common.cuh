@@ -29,6 +29,7 @@ struct LhDims {
   int nPartial;  // levels 0..nPartial-1 are partially selected (k < N_l); the rest are kept whole
   int Nl[LH_MAX_LEVELS];     // entries of level l
   int wl[LH_MAX_LEVELS];     // tokens per entry of level l
+  int wlog[LH_MAX_LEVELS];   // log2(wl[l]) (windows are powers of two for every supported p)
   int off[LH_MAX_LEVELS];    // global pyramid id (= slot row) of entry (l, 0)
   int poff[LH_MAX_LEVELS];   // row of level l (>= 1) inside the per-head pyramid of lh_pool
   int kl[LH_MAX_LEVELS];     // selected entries of level l

@@ -129,6 +129,16 @@ template <int D, int P, int LEV>
 __device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8]) {
   if constexpr (LEV == 0) {
     load_row8(ld16(p), out);
+  } else if constexpr (ipow(P, LEV) <= 16) {
+    // few enough rows to keep all of their loads in flight at once; the sums keep the tree order
+    constexpr int CW = ipow(P, LEV - 1);
+#pragma unroll
+    for (int c = 0; c < P; ++c) {
+      double ch[8];
+      tree_sum<D, P, LEV - 1>(p + (int64_t)c * CW * D, ch);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? ch[i] : out[i] + ch[i];
+    }
   } else {
     constexpr int CW = ipow(P, LEV - 1);
 #pragma unroll 1

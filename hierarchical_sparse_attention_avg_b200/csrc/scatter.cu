@@ -68,28 +68,88 @@ __device__ __forceinline__ float head_scale(float amax) {
   return ldexpf(1.f, 10 - e);
 }
 
+// Tokens per row group in the token-major kernels: every slot lookup of the group is issued before any row load,
+// so a thread keeps up to kMaxL * kTok independent loads in flight instead of a chain of dependent ones.
+constexpr int kTok = 4;
+constexpr int kMaxL = 5;
+
+// Row group g covers the kTok tokens whose "key" is g*kTok .. g*kTok + kTok - 1, where key = t + 1 for the offset
+// scatter (entry j = key/w - 1) and key = t for the unpool (j = key/w).  Windows are powers of two, so for every
+// level with w >= kTok the whole group reads ONE entry (one slot lookup, one row load, added to all kTok tokens);
+// only narrower levels need per-token lookups.  Rows are summed in fp32 with per-level weights.
+template <int D, bool kOffset>
+__device__ __forceinline__ void token_sum(const float* __restrict__ src, const int32_t* __restrict__ sl, int bh,
+                                          int key0, int lane, const LhDims& dm, float (&acc)[kTok][8]) {
+  int s[kMaxL][kTok];
+#pragma unroll
+  for (int lev = 0; lev < kMaxL; ++lev) {
+#pragma unroll
+    for (int u = 0; u < kTok; ++u) s[lev][u] = -1;
+    if (lev >= dm.L) continue;
+    const int sh = dm.wlog[lev];
+    if ((1 << sh) >= kTok) {
+      const int j = (key0 >> sh) - (kOffset ? 1 : 0);
+      if (j >= 0 && j < dm.Nl[lev]) s[lev][0] = sl[dm.off[lev] + j];
+    } else {
+#pragma unroll
+      for (int u = 0; u < kTok; ++u) {
+        const int j = ((key0 + u) >> sh) - (kOffset ? 1 : 0);
+        if (j >= 0 && j < dm.Nl[lev]) s[lev][u] = sl[dm.off[lev] + j];
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kTok; ++u)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+#pragma unroll
+  for (int lev = 0; lev < kMaxL; ++lev) {
+    if (lev >= dm.L) continue;
+    const int sh = dm.wlog[lev];
+    const float wgt = kOffset ? 1.0f : __uint_as_float((127u - (uint32_t)sh) << 23);  // 2^-sh, exact
+    if ((1 << sh) >= kTok) {
+      if (s[lev][0] >= 0) {
+        float f[8];
+        load8f(src + ((int64_t)bh * dm.S + s[lev][0]) * D + lane * 8, f);
+#pragma unroll
+        for (int u = 0; u < kTok; ++u)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(f[i], wgt, acc[u][i]);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kTok; ++u) {
+        if (s[lev][u] >= 0) {
+          float f[8];
+          load8f(src + ((int64_t)bh * dm.S + s[lev][u]) * D + lane * 8, f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(f[i], wgt, acc[u][i]);
+        }
+      }
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) scatter_kernel(const float* __restrict__ og, const int32_t* __restrict__ slot,
                                                       __nv_bfloat16* __restrict__ o, LhDims dm) {
   constexpr int G = D / 8;
   const int lane = threadIdx.x % G;
-  const int64_t row = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
-  if (row >= (int64_t)dm.BH * dm.N) return;
-  const int bh = (int)(row / dm.N);
-  const int t = (int)(row % dm.N);
-  const int32_t* sl = slot + (int64_t)bh * dm.R;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int lev = 0; lev < dm.L; ++lev) {
-    const int j = (t + 1) / dm.wl[lev] - 1;
-    if (j < 0) continue;
-    const int s = sl[dm.off[lev] + j];
-    if (s < 0) continue;
-    float f[8];
-    load8f(og + ((int64_t)bh * dm.S + s) * D + lane * 8, f);
+  const int gph = (dm.N + kTok) / kTok;  // row groups per head: keys t + 1 = 1 .. N
+  const int64_t ngrp = (int64_t)dm.BH * gph;
+  // grid-stride over row groups: a few resident blocks per SM instead of one short-lived block per 64 tokens
+  for (int64_t grp = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G; grp < ngrp;
+       grp += (int64_t)gridDim.x * (256 / G)) {
+    const int bh = (int)(grp / gph);
+    const int key0 = (int)(grp % gph) * kTok;
+    float acc[kTok][8];
+    token_sum<D, true>(og, slot + (int64_t)bh * dm.R, bh, key0, lane, dm, acc);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += f[i];
+    for (int u = 0; u < kTok; ++u) {
+      const int t = key0 + u - 1;
+      if (t >= 0 && t < dm.N) st_stream16(o + ((int64_t)bh * dm.N + t) * D + lane * 8, pack8_rn(acc[u]));
+    }
   }
-  st_stream16(o + row * D + lane * 8, pack8_rn(acc));
 }
 
 // One group per gathered row: dog[s] = fp32 window sum of dout.  With amax non-null, also the running per-head
@@ -207,24 +267,20 @@ __global__ void __launch_bounds__(256) unpool_bwd_kernel(const float* __restrict
   constexpr int G = D / 8;
   const int which = blockIdx.y;
   const int lane = threadIdx.x % G;
-  const int64_t row = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
-  if (row >= (int64_t)dm.BH * dm.N) return;
-  const int bh = (int)(row / dm.N);
-  const int t = (int)(row % dm.N);
-  const int32_t* sl = slot + (int64_t)bh * dm.R;
+  const int gph = (dm.N + kTok - 1) / kTok;
+  const int64_t ngrp = (int64_t)dm.BH * gph;
   const float* src = which == 0 ? dqg : (which == 1 ? dkg : dvg);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int lev = 0; lev < dm.L; ++lev) {
-    const int s = sl[dm.off[lev] + t / dm.wl[lev]];
-    if (s < 0) continue;
-    const float inv_w = 1.0f / (float)dm.wl[lev];  // exact: power-of-two window
-    float f[8];
-    load8f(src + ((int64_t)bh * dm.S + s) * D + lane * 8, f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = fmaf(f[i], inv_w, acc[i]);
-  }
   __nv_bfloat16* out = which == 0 ? dq : (which == 1 ? dk : dv);
-  st_stream16(out + row * D + lane * 8, pack8_rn(acc));
+  for (int64_t grp = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G; grp < ngrp;
+       grp += (int64_t)gridDim.x * (256 / G)) {
+    const int bh = (int)(grp / gph);
+    const int t0 = (int)(grp % gph) * kTok;  // key = t
+    float acc[kTok][8];
+    token_sum<D, false>(src, slot + (int64_t)bh * dm.R, bh, t0, lane, dm, acc);
+#pragma unroll
+    for (int u = 0; u < kTok; ++u)
+      if (t0 + u < dm.N) st_stream16(out + ((int64_t)bh * dm.N + t0 + u) * D + lane * 8, pack8_rn(acc[u]));
+  }
 }
 
 template <int D>
@@ -232,15 +288,33 @@ int blocks_for(int64_t rows) {
   return (int)((rows + 256 / (D / 8) - 1) / (256 / (D / 8)));
 }
 
+// Blocks for a grid-stride kernel: enough for every row group, capped at what the device keeps resident at once
+// (blocks per SM from the occupancy calculator times the SM count), so the loop has no ragged last wave.
+template <typename Kernel>
+int resident_blocks(Kernel kernel, int64_t need) {
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0);
+  const int64_t cap = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+  return (int)(need < cap ? need : cap);
+}
+
+// `slices` launches share the device (gridDim.y), so each gets 1/slices of the resident blocks.
+template <int D, typename Kernel>
+int token_blocks(Kernel kernel, const LhDims& dm, int slices) {
+  const int b = resident_blocks(kernel, blocks_for<D>((int64_t)dm.BH * ((dm.N + kTok - 1) / kTok))) / slices;
+  return b > 0 ? b : 1;
+}
+
 }  // namespace
 
 int launch_scatter(const float* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st) {
-  const int64_t rows = (int64_t)dm.BH * dm.N;
   KernelTimer timer("scatter", st);
   if (dm.d == 64)
-    scatter_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
+    scatter_kernel<64><<<token_blocks<64>(scatter_kernel<64>, dm, 1), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
   else
-    scatter_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
+    scatter_kernel<128><<<token_blocks<128>(scatter_kernel<128>, dm, 1), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
   return check_launch();
 }
 
@@ -278,13 +352,12 @@ int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax,
 
 int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st) {
-  const int64_t rows = (int64_t)dm.BH * dm.N;
   KernelTimer timer("unpool_bwd", st);
   if (dm.d == 64)
-    unpool_bwd_kernel<64><<<dim3(blocks_for<64>(rows), 3), 256, 0, st>>>(
+    unpool_bwd_kernel<64><<<dim3(token_blocks<64>(unpool_bwd_kernel<64>, dm, 3), 3), 256, 0, st>>>(
         dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
   else
-    unpool_bwd_kernel<128><<<dim3(blocks_for<128>(rows), 3), 256, 0, st>>>(
+    unpool_bwd_kernel<128><<<dim3(token_blocks<128>(unpool_bwd_kernel<128>, dm, 3), 3), 256, 0, st>>>(
         dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
   return check_launch();
 }
