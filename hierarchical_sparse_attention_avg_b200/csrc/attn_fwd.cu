@@ -4,53 +4,56 @@
 // standard scaled-dot-product attention the pages run on the gathered rows ([W] 核心方法 §3 标准 FlashAttention
 // 调用; [H] "How Lighthouse Attention Works").  The pages call a library kernel here; this is a kernel of its own.
 //
-// One CTA (128 threads) per (head, 128-row query tile), heaviest tiles first.  For each 128-row key tile:
-//   TMA (128-byte swizzle) brings K_j and V_j into a two-stage ring while the previous tile computes;
-//   one thread issues S = Q K_j^T (tcgen05.mma, M = N = 128, fp32 accumulator in tensor memory);
-//   every thread owns one query row = one TMEM lane: it reads its 128 scores, applies the causal mask on the
-//   diagonal tile, updates the running max (O in tensor memory is rescaled when any row of the warp grows),
-//   exponentiates in base 2 and writes P (bf16) into a swizzled shared-memory tile.  Keeping the reference at
-//   the running max makes the dominant key's P exactly 1, so O = P V stays consistent with the fp32 P the
-//   backward recomputes (D = rowsum(dO o O) then matches sum_b P dP);
-//   one thread issues O += P V_j (A = P K-major, B = V_j MN-major, fp32 accumulator in tensor memory).
-// O_g is written in fp32: the backward's D and the scatter-back read it at full accumulator precision.
-// Every wait is bounded; a timeout records LH_ERR_TIMEOUT and the block leaves after draining its own copies
-// and MMAs.
+// One CTA per (head, 128-row query tile), heaviest tiles first, with warp roles:
+//   warp 0     TMA producer: Q once; K_j and V_j into two-stage rings with their own full/empty barriers;
+//   warp 1     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM score buffers, then O_b += P_j V_j;
+//   warps 2-5  softmax, one query row (= one TMEM lane) per thread.
+// The MMA thread issues S_{j+1} before O += P_j V_j, so the tensor core computes the next scores while the
+// softmax works on the current ones.  There are two O accumulators in tensor memory: tile j accumulates into O_b,
+// b = j mod 2, so before the softmax rescales O_b to its new running max and overwrites P buffer b it only waits
+// for the product of tile j-2 (long finished in steady state).  At the end the two accumulators are brought to
+// the final max and added.  The reference max is always the running max itself, so the dominant key's P is
+// exactly 1 and O = P V stays consistent with the fp32 P the backward recomputes; O_g is stored in fp32.
+// Operands are fp16 (Q, K, V exact from their bf16 values; P in [0, 1]); accumulators fp32.
+// Every wait is bounded; a timeout records LH_ERR_TIMEOUT and every role leaves after draining its own work.
 #include "internal.h"
 
 namespace lh {
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kTile = 128;                 // query rows and key rows per tile
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kThreads = 192;
+constexpr int kTile = 128;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct FwdLayout {
-  static constexpr uint32_t TILE = kTile * D * 2;  // bytes of one [128][D] bf16 tile (D/64 swizzled blocks)
+  static constexpr uint32_t TILE = kTile * D * 2;  // one [128][D] fp16 tile (D/64 swizzled 16 KB blocks)
+  static constexpr uint32_t PT = kTile * kTile * 2;  // one [128][128] fp16 P tile
   static constexpr uint32_t Q = 0;
-  static constexpr uint32_t K = TILE;              // two stages
-  static constexpr uint32_t V = 3 * TILE;          // two stages
-  static constexpr uint32_t P = 5 * TILE;          // [128][128] bf16, two 64-column swizzled blocks
-  static constexpr uint32_t BAR = P + kTile * kTile * 2;
-  static constexpr uint32_t BYTES = BAR + 128;
+  static constexpr uint32_t K = TILE;              // 2 stages
+  static constexpr uint32_t V = 3 * TILE;          // 2 stages
+  static constexpr uint32_t P = 5 * TILE;          // 2 buffers
+  static constexpr uint32_t BAR = P + 2 * PT;
+  // barriers (8 bytes each)
+  static constexpr uint32_t B_Q = 0, B_KF = 1, B_KE = 3, B_VF = 5, B_VE = 7, B_SF = 9, B_SE = 11, B_PF = 13,
+                            B_OD = 15, B_DRAIN = 17, NBAR = 18;
+  static constexpr uint32_t BYTES = BAR + NBAR * 8;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, float* __restrict__ og,
-                    float* __restrict__ lse, int S, int ntiles, float scale_log2, int* status) {
+                    const __grid_constant__ CUtensorMap tmV, float* __restrict__ og, float* __restrict__ lse, int S,
+                    int ntiles, float scale_log2, int* status) {
   using Lay = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_q = sb + Lay::BAR, bar_kv0 = bar_q + 8, bar_s = bar_q + 24, bar_o = bar_q + 32;
-  const uint32_t bar_drain = bar_q + 40;
+  auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qt = ntiles - 1 - (int)blockIdx.x;  // heaviest query tiles first
@@ -59,183 +62,230 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    mbar_init(bar_q, 1);
-    mbar_init(bar_kv0, 1);
-    mbar_init(bar_kv0 + 8, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar(Lay::B_Q), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(Lay::B_KF + b), 1);
+      mbar_init(bar(Lay::B_KE + b), 1);
+      mbar_init(bar(Lay::B_VF + b), 1);
+      mbar_init(bar(Lay::B_VE + b), 1);
+      mbar_init(bar(Lay::B_SF + b), 1);
+      mbar_init(bar(Lay::B_SE + b), kTile);
+      mbar_init(bar(Lay::B_PF + b), kTile);
+      mbar_init(bar(Lay::B_OD + b), 1);
+    }
+    mbar_init(bar(Lay::B_DRAIN), 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
-  if (warp == 0) tmem_alloc(smem_u32(&s_tmem), 256);
+  if (warp == 1) tmem_alloc(smem_u32(&s_tmem), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem;        // columns [0, 128): scores
-  const uint32_t tO = tmem + 128;  // columns [128, 128 + D): output accumulator
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t tmem = s_tmem;  // columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D)
 
-  constexpr uint32_t idesc_qk = idesc_f32acc(kFmtF16, 128, 128, 0, 0);
-  constexpr uint32_t idesc_pv = idesc_f32acc(kFmtF16, 128, D, 0, 1);
-
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_q, Lay::TILE);
-    for (int db = 0; db < D / 64; ++db) tma_load_3d(sb + Lay::Q + db * 16384, &tmQ, bar_q, db * 64, qt * kTile, bh);
-    mbar_arrive_expect_tx(bar_kv0, 2 * Lay::TILE);
-    for (int db = 0; db < D / 64; ++db) {
-      tma_load_3d(sb + Lay::K + db * 16384, &tmK, bar_kv0, db * 64, 0, bh);
-      tma_load_3d(sb + Lay::V + db * 16384, &tmV, bar_kv0, db * 64, 0, bh);
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int kv_issued = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(bar(Lay::B_Q), Lay::TILE);
+      for (int db = 0; db < D / 64; ++db)
+        tma_load_3d(sb + Lay::Q + db * 16384, &tmQ, bar(Lay::B_Q), db * 64, qt * kTile, bh);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int b = j & 1;
+        const uint32_t ph = ((j >> 1) - 1) & 1;  // phase of the previous use of this stage
+        if (j >= 2) ok = mbar_wait(bar(Lay::B_KE + b), ph, &s_abort, status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(Lay::B_KF + b), Lay::TILE);
+        for (int db = 0; db < D / 64; ++db)
+          tma_load_3d(sb + Lay::K + b * Lay::TILE + db * 16384, &tmK, bar(Lay::B_KF + b), db * 64, j * kTile, bh);
+        if (j >= 2) ok = mbar_wait(bar(Lay::B_VE + b), ph, &s_abort, status);
+        if (!ok) {
+          kv_issued = j;  // K_j in flight without its V
+          mbar_wait_teardown(bar(Lay::B_KF + b), (j >> 1) & 1);
+          break;
+        }
+        mbar_arrive_expect_tx(bar(Lay::B_VF + b), Lay::TILE);
+        for (int db = 0; db < D / 64; ++db)
+          tma_load_3d(sb + Lay::V + b * Lay::TILE + db * 16384, &tmV, bar(Lay::B_VF + b), db * 64, j * kTile, bh);
+        kv_issued = j + 1;
+      }
+      if (!ok) {  // drain the copies this thread issued before leaving
+        mbar_wait_teardown(bar(Lay::B_Q), 0);
+        for (int j = kv_issued >= 2 ? kv_issued - 2 : 0; j < kv_issued; ++j) {
+          mbar_wait_teardown(bar(Lay::B_KF + (j & 1)), (j >> 1) & 1);
+          mbar_wait_teardown(bar(Lay::B_VF + (j & 1)), (j >> 1) & 1);
+        }
+      }
     }
-  }
-
-  const int row = warp * 32 + lane;  // query row inside the tile = TMEM lane
-  float m_run = -INFINITY, l_run = 0.f;
-  int issued_kv = 1;                 // K/V tiles whose loads were issued
-  bool ok = true;
-
-  for (int j = 0; j < nkv && ok; ++j) {
-    const int st = j & 1;
-    const uint32_t sK = sb + Lay::K + st * Lay::TILE, sV = sb + Lay::V + st * Lay::TILE;
-    if (threadIdx.x == 0) {
-      bool got = (j > 0 || mbar_wait(bar_q, 0, &s_abort, status)) &&
-                 mbar_wait(bar_kv0 + 8 * st, (j >> 1) & 1, &s_abort, status);
-      if (got) {
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f32acc(kFmtF16, 128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_f32acc(kFmtF16, 128, D, 0, 1);
+      bool ok = mbar_wait(bar(Lay::B_Q), 0, &s_abort, status);
+      auto issue_pv = [&](int jp) {
+        const int bp = jp & 1;
+        const uint32_t php = (jp >> 1) & 1;
+        if (!mbar_wait(bar(Lay::B_VF + bp), php, &s_abort, status)) return false;
+        if (!mbar_wait(bar(Lay::B_PF + bp), php, &s_abort, status)) return false;
         tc_fence_after();
+        const uint32_t tO = tmem + 256 + 128 * bp;
+        const uint32_t sP = sb + Lay::P + bp * Lay::PT, sV = sb + Lay::V + bp * Lay::TILE;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ss(tO, sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv, (jp >= 2 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(Lay::B_OD + bp));
+        umma_commit(bar(Lay::B_VE + bp));
+        return true;
+      };
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        ok = mbar_wait(bar(Lay::B_KF + b), ph, &s_abort, status);
+        if (ok && j >= 2) ok = mbar_wait(bar(Lay::B_SE + b), ph ^ 1, &s_abort, status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tmem + 128 * b;
+        const uint32_t sK = sb + Lay::K + b * Lay::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
           umma_ss(tS, sdesc_sw128(sb + Lay::Q + koff, 16, 1024), sdesc_sw128(sK + koff, 16, 1024), idesc_qk,
-                       kk > 0);
+                  kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar_s);
-        if (j + 1 < nkv) {  // the other stage was released by the PV product of tile j-1 (waited below)
-          const uint32_t bar = bar_kv0 + 8 * (st ^ 1);
-          const uint32_t sK2 = sb + Lay::K + (st ^ 1) * Lay::TILE, sV2 = sb + Lay::V + (st ^ 1) * Lay::TILE;
-          mbar_arrive_expect_tx(bar, 2 * Lay::TILE);
-          for (int db = 0; db < D / 64; ++db) {
-            tma_load_3d(sK2 + db * 16384, &tmK, bar, db * 64, (j + 1) * kTile, bh);
-            tma_load_3d(sV2 + db * 16384, &tmV, bar, db * 64, (j + 1) * kTile, bh);
+        umma_commit(bar(Lay::B_SF + b));
+        umma_commit(bar(Lay::B_KE + b));
+        if (j >= 1) ok = issue_pv(j - 1);
+      }
+      if (ok) issue_pv(nkv - 1);
+      // drain: every product issued above completes before the block releases its memory
+      umma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_teardown(bar(Lay::B_DRAIN), 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    float m_ref[2] = {-INFINITY, -INFINITY};
+    bool ok = true;
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int b = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), ph, &s_abort, status));  // warp-uniform
+      if (!ok) break;
+      tc_fence_after();
+      float s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + 128 * b + lane_base + c * 32, s[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_SE + b));  // score buffer b may be overwritten by S_{j+2}
+
+      const bool diag = (j == qt);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float x = s[c][i] * scale_log2;
+          if (diag && (c * 32 + i) > row) x = -INFINITY;
+          s[c][i] = x;
+          mx = fmaxf(mx, x);
+        }
+      const float m_new = fmaxf(m_run, mx);
+      l_run *= ex2(m_run - m_new);  // 1 without growth; 0 on the first tile
+      m_run = m_new;
+      // P of this tile (fp16, in [0, 1]) and its row sum
+      uint32_t pk[64];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2(s[c][i] - m_run), p1 = ex2(s[c][i + 1] - m_run);
+          rs += p0 + p1;
+          pk[c * 16 + i / 2] = pack_half2_rn(p0, p1);
+        }
+      l_run += rs;
+      // O_b and P buffer b are free once the product of tile j-2 has completed
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_OD + b), ph ^ 1, &s_abort, status));
+        if (!ok) break;
+        tc_fence_after();
+        const float alpha = ex2(m_ref[b] - m_run);
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          const uint32_t tO = tmem + 256 + 128 * b + lane_base;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + c * 32, o);
           }
-          issued_kv = j + 2;
+          tmem_st_wait();
         }
-      } else {
-        s_abort = 1;
       }
-    }
-    ok = mbar_wait(bar_s, j & 1, &s_abort, status);
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-
-    float s[4][32];
+      m_ref[b] = m_run;
+      uint8_t* sP = smem + Lay::P + b * Lay::PT;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_base + c * 32, s[c]);
-    tmem_ld_wait();
-
-    const bool diag = (j == qt);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float x = s[c][i] * scale_log2;
-        if (diag && (c * 32 + i) > row) x = -INFINITY;
-        s[c][i] = x;
-        mx = fmaxf(mx, x);
+      for (int ch = 0; ch < 16; ++ch) {  // 16-byte chunk ch holds keys 8*ch .. 8*ch+7
+        const uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+        *reinterpret_cast<uint4*>(sP + (ch >> 3) * 16384 + sw128_offset(row, ch & 7)) = v;
       }
-    const bool grow = mx > m_run;
-    const float m_new = grow ? mx : m_run;
-    const float alpha = ex2(m_run - m_new);  // 1 without growth; 0 on the first tile
-    if (j > 0 && __any_sync(0xffffffffu, grow)) {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_PF + b));
+    }
+    // epilogue: wait for the last products, bring both accumulators to the final max, normalise, store
+    if (ok) {
+      const int jl = nkv - 1;
+      ok = mbar_wait(bar(Lay::B_OD + (jl & 1)), (jl >> 1) & 1, &s_abort, status);
+      if (ok && nkv >= 2) ok = mbar_wait(bar(Lay::B_OD + ((jl - 1) & 1)), ((jl - 1) >> 1) & 1, &s_abort, status);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      const float a0 = ex2(m_ref[0] - m_run) * inv_l;
+      const float a1 = nkv >= 2 ? ex2(m_ref[1] - m_run) * inv_l : 0.f;
+      const int grow_idx = qt * kTile + row;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(tO + lane_base + c * 32, o);
+        float o0[32], o1[32];
+        tmem_ld32(tmem + 256 + lane_base + c * 32, o0);
+        tmem_ld32(tmem + 384 + lane_base + c * 32, o1);
         tmem_ld_wait();
+        if (grow_idx < S) {
+          float4* dst = reinterpret_cast<float4*>(og + ((int64_t)bh * S + grow_idx) * D + c * 32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-        tmem_st32(tO + lane_base + c * 32, o);
-      }
-      tmem_st_wait();
-    }
-    m_run = m_new;
-    float rs = 0.f;
-    uint8_t* sP = smem + Lay::P;
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float r[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          p[i] = ex2(s[c][q8 * 8 + i] - m_run);
-          rs += p[i];
+            for (int e = 0; e < 4; ++e) {
+              const int i = q4 * 4 + e;
+              r[e] = nkv >= 2 ? fmaf(o0[i], a0, o1[i] * a1) : o0[i] * a0;
+            }
+            dst[q4] = make_float4(r[0], r[1], r[2], r[3]);
+          }
         }
-        const int col = c * 32 + q8 * 8;  // first key column of this 16-byte chunk
-        const uint4 v = make_uint4(pack_half2_rn(p[0], p[1]), pack_half2_rn(p[2], p[3]),
-                                   pack_half2_rn(p[4], p[5]), pack_half2_rn(p[6], p[7]));
-        *reinterpret_cast<uint4*>(sP + (col >> 6) * 16384 + sw128_offset(row, (col & 63) >> 3)) = v;
       }
+      if (grow_idx < S) lse[(int64_t)bh * S + grow_idx] = (m_run + __log2f(l_run)) * kLn2;
     }
-    l_run = l_run * alpha + rs;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        const uint64_t a = sdesc_sw128(sb + Lay::P + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t b = sdesc_sw128(sV + kk * 2048, 16384, 1024);
-        umma_ss(tO, a, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-      }
-      umma_commit(bar_o);
-    }
-    ok = mbar_wait(bar_o, j & 1, &s_abort, status);
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
   }
 
-  if (ok) {
-    const int grow_idx = qt * kTile + row;
-    const float inv_l = 1.0f / l_run;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      tmem_ld32(tO + lane_base + c * 32, o);
-      tmem_ld_wait();
-      if (grow_idx < S) {
-        float4* dst = reinterpret_cast<float4*>(og + ((int64_t)bh * S + grow_idx) * D + c * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          dst[q4] = make_float4(o[q4 * 4 + 0] * inv_l, o[q4 * 4 + 1] * inv_l, o[q4 * 4 + 2] * inv_l,
-                                o[q4 * 4 + 3] * inv_l);
-      }
-    }
-    if (grow_idx < S) lse[(int64_t)bh * S + grow_idx] = (m_run + __log2f(l_run)) * kLn2;
-  } else if (threadIdx.x == 0) {
-    // drain: outstanding TMA copies and MMAs must finish before shared and tensor memory are released
-    umma_commit(bar_drain);
-    mbar_wait_teardown(bar_drain, 0);
-    mbar_wait_teardown(bar_q, 0);
-    // only the last two K/V tiles can still be in flight, one per stage (older phases were consumed)
-    for (int t = issued_kv >= 2 ? issued_kv - 2 : 0; t < issued_kv; ++t)
-      mbar_wait_teardown(bar_kv0 + 8 * (t & 1), (t >> 1) & 1);
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -252,8 +302,7 @@ int launch_fwd_t(const void* qg, const void* kg, const void* vg, float* og, floa
   const int nt = (dm.S + kTile - 1) / kTile;
   const float scale_log2 = kLog2e / sqrtf((float)D);
   KernelTimer timer("attn_fwd", st);
-  attn_fwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, nt,
-                                                               scale_log2, dm.status);
+  attn_fwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, nt, scale_log2, dm.status);
   return check_launch();
 }
 
