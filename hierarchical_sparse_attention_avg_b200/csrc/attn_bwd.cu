@@ -5,266 +5,325 @@
 // leave this to the attention library's autograd ([W] 深度洞察; [E] "Как four-stage pipeline…"); this is a kernel
 // of its own.
 //
-// One CTA (128 threads) per (head, 128-row key tile); K_j, V_j stay in shared memory while the query tiles
-// i >= j stream through (TMA, 128-byte swizzle).  Per query tile:
-//   S^T = K_j Q_i^T and dP^T = V_j dO_i^T (tensor memory, M = 128 key rows, N = 128 query rows);
-//   each thread owns one key row (one TMEM lane): P^T and dS^T rows go to swizzled shared-memory tiles (bf16);
-//   dV_j += P^T dO_i and dK_j += dS^T Q_i accumulate in tensor memory for the whole loop;
-//   dQ_i^T = K_j^T dS^T (M = 128 over the head dimension, N = 128 query rows) lands in the S^T columns, and each
-//   thread (one feature) adds its 128 values to the fp32 dQ accumulator in global memory: a warp's 32 lanes
-//   touch 32 consecutive floats of one row, so every atomic instruction is one coalesced 128-byte reduction.
-// For d = 64 the dQ^T product still uses M = 128; lanes 64..127 are ignored.
+// One CTA per (head, 128-row key tile); K_j and V_j stay in shared memory while the 64-row query sub-tiles i that
+// can see them (64 i + 63 >= 128 j) stream through.  Warp roles:
+//   warp 0     TMA producer: K_j, V_j once; Q_i and dO_i into a two-stage ring;
+//   warp 1     MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into one of two TMEM buffer pairs,
+//              then, for the previous sub-tile, dV += P^T dO, dK += dS^T Q (accumulated in TMEM for the whole
+//              loop) and dQ^T = K_j^T dS^T (into the consumed S^T columns);
+//   warps 2-5  compute: one key row (TMEM lane) per thread writes the P^T and dS^T rows (fp16) of the sub-tile;
+//   warps 6-9  drain: one feature (TMEM lane) per thread moves dQ^T out of TMEM into a shared-memory tile that
+//              one thread adds to the fp32 dQ accumulator with TMA bulk tensor reduce-add.
+// The MMA thread issues S^T/dP^T of sub-tile i+1 before the products of sub-tile i, so the tensor core works while
+// the compute warps do.  64-row sub-tiles keep the double-buffered S^T/dP^T (4 x 64 columns) and the dV/dK
+// accumulators (2 x d columns) inside the 512 tensor-memory columns.
 // Operands are fp16 (gathered Q, K, V exactly; P in [0, 1]; dO_g and dS scaled per head by a power of two so
-// that their largest magnitudes sit near 2^10): the layer's window-summed dO_g makes the dS and dV sums cancel
-// strongly, and bf16 operands (8-bit significands) were measured to exceed the 2e-2 + 2e-2|ref| tolerance where
-// fp16 (11-bit) stays within it at the same tensor-core rate.  Results are multiplied by the inverse scale; a
-// dS beyond the fp16 range records LH_ERR_RANGE.
+// their largest magnitudes sit near 2^10): the layer's window-summed dO_g makes dS and dV sums cancel strongly,
+// and bf16 operands were measured to exceed the 2e-2 + 2e-2|ref| tolerance where fp16 stays within it.  Results
+// are multiplied by the inverse scale; a dS beyond the fp16 range records LH_ERR_RANGE.  For d = 64 the dQ^T
+// product still uses M = 128 (lanes 64..127 ignored).  Every wait is bounded.
 #include "internal.h"
 
 namespace lh {
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kTile = 128;
+constexpr int kThreads = 320;
+constexpr int kKTile = 128;  // key rows per CTA
+constexpr int kQTile = 64;   // query rows per sub-tile
+constexpr int kStages = 2;   // Q/dO ring depth
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kBarCompute = 1, kBarDrain = 2;  // named barrier ids (0 is __syncthreads)
 
 template <int D>
 struct BwdLayout {
-  static constexpr uint32_t TILE = kTile * D * 2;
+  static constexpr uint32_t KT = kKTile * D * 2;       // K or V tile
+  static constexpr uint32_t QT = kQTile * D * 2;       // Q or dO sub-tile (d-blocks of 8 KB)
+  static constexpr uint32_t PT = kKTile * kQTile * 2;  // P^T or dS^T tile: 128 rows x 128 bytes (16 KB)
   static constexpr uint32_t K = 0;
-  static constexpr uint32_t V = TILE;
-  static constexpr uint32_t Q = 2 * TILE;
-  static constexpr uint32_t DO = 3 * TILE;
-  static constexpr uint32_t P = 4 * TILE;              // [128 key][128 query] bf16, two swizzled blocks
-  static constexpr uint32_t DS = P + kTile * kTile * 2;
-  static constexpr uint32_t LSE = DS + kTile * kTile * 2;  // 128 fp32: LSE * log2(e) of the query tile
-  static constexpr uint32_t DV = LSE + 512;                // 128 fp32: D of the query tile
-  static constexpr uint32_t BAR = DV + 512;
-  static constexpr uint32_t BYTES = BAR + 128;
+  static constexpr uint32_t V = KT;
+  static constexpr uint32_t Q = 2 * KT;                      // kStages
+  static constexpr uint32_t DO = Q + kStages * QT;           // kStages
+  static constexpr uint32_t P = DO + kStages * QT;           // 2 buffers
+  static constexpr uint32_t DS = P + 2 * PT;                 // 2 buffers
+  static constexpr uint32_t DQ = DS + 2 * PT;                // staging: [d/32][64 q][32 f] fp32
+  static constexpr uint32_t STAT = DQ + kQTile * D * 4;      // [2][64] LSE*log2e, [2][64] D
+  static constexpr uint32_t BAR = STAT + 4 * kQTile * 4;
+  static constexpr uint32_t B_KV = 0, B_QF = 1, B_QE = 1 + kStages, B_SF = 1 + 2 * kStages, B_DSF = B_SF + 2,
+                            B_MM = B_DSF + 2, B_DQF = B_MM + 2, B_FIN = B_DQF + 2, B_DRAIN = B_FIN + 1,
+                            NBAR = B_DRAIN + 1;
+  static constexpr uint32_t BYTES = BAR + NBAR * 8;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const float* __restrict__ lse, const float* __restrict__ dvec, const float* __restrict__ dinv,
-                    float* __restrict__ dqacc, float* __restrict__ dkg, float* __restrict__ dvg, int S, int ntiles,
-                    float scale, int* status) {
+                    const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
+                    const float* __restrict__ dvec, const float* __restrict__ dinv, float* __restrict__ dkg,
+                    float* __restrict__ dvg, int S, float scale, int* status) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_kv = sb + Lay::BAR, bar_qd = bar_kv + 8, bar_mm1 = bar_kv + 16, bar_mm2 = bar_kv + 24;
-  const uint32_t bar_drain = bar_kv + 32;
-  float* s_lse = reinterpret_cast<float*>(smem + Lay::LSE);
-  float* s_d = reinterpret_cast<float*>(smem + Lay::DV);
+  auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int kt = blockIdx.x;  // key tile: tile 0 meets the most query tiles and is scheduled first
+  const int kt = blockIdx.x;  // key tile: tile 0 meets the most query sub-tiles and is scheduled first
   const int bh = blockIdx.y;
+  const int nq = (S + kQTile - 1) / kQTile;
+  const int i0 = 2 * kt;  // first sub-tile with a query at or after the tile's first key
+  const int nit = nq - i0;
   const float scale_log2 = scale * kLog2e;
+  const float inv_scale = dinv[bh];
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    mbar_init(bar_kv, 1);
-    mbar_init(bar_qd, 1);
-    mbar_init(bar_mm1, 1);
-    mbar_init(bar_mm2, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar(Lay::B_KV), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(Lay::B_QF + s), 1);
+      mbar_init(bar(Lay::B_QE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(Lay::B_SF + b), 1);
+      mbar_init(bar(Lay::B_DSF + b), 128);
+      mbar_init(bar(Lay::B_MM + b), 1);
+      mbar_init(bar(Lay::B_DQF + b), 128);
+    }
+    mbar_init(bar(Lay::B_FIN), 1);
+    mbar_init(bar(Lay::B_DRAIN), 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmDO);
+    prefetch_tmap(&tmDQ);
   }
-  if (warp == 0) tmem_alloc(smem_u32(&s_tmem), 512);
+  if (warp == 1) tmem_alloc(smem_u32(&s_tmem), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem;            // S^T, later dQ^T
-  const uint32_t tDP = tmem + 128;     // dP^T
-  const uint32_t tDV = tmem + 256;     // dV accumulator (D columns)
-  const uint32_t tDK = tmem + 256 + D; // dK accumulator (D columns)
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  // columns: S^T buffer b at 128 b, dP^T buffer b at 128 b + 64; dV at 256; dK at 256 + D
+  const uint32_t tDV = tmem + 256, tDK = tmem + 256 + D;
 
-  constexpr uint32_t idesc_kk = idesc_f32acc(kFmtF16, 128, 128, 0, 0);  // both operands K-major
-  constexpr uint32_t idesc_acc = idesc_f32acc(kFmtF16, 128, D, 0, 1);   // A K-major, B MN-major
-  constexpr uint32_t idesc_dq = idesc_f32acc(kFmtF16, 128, 128, 1, 1);  // both operands MN-major
-  const float inv_scale = dinv[bh];                                     // undoes the per-head dO_g scale
-
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_kv, 2 * Lay::TILE);
-    for (int db = 0; db < D / 64; ++db) {
-      tma_load_3d(sb + Lay::K + db * 16384, &tmK, bar_kv, db * 64, kt * kTile, bh);
-      tma_load_3d(sb + Lay::V + db * 16384, &tmV, bar_kv, db * 64, kt * kTile, bh);
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      mbar_arrive_expect_tx(bar(Lay::B_KV), 2 * Lay::KT);
+      for (int db = 0; db < D / 64; ++db) {
+        tma_load_3d(sb + Lay::K + db * 16384, &tmK, bar(Lay::B_KV), db * 64, kt * kKTile, bh);
+        tma_load_3d(sb + Lay::V + db * 16384, &tmV, bar(Lay::B_KV), db * 64, kt * kKTile, bh);
+      }
+      for (int it = 0; it < nit && ok; ++it) {
+        const int s = it % kStages;
+        if (it >= kStages) ok = mbar_wait(bar(Lay::B_QE + s), ((it / kStages) - 1) & 1, &s_abort, status);
+        if (!ok) break;
+        const int row = (i0 + it) * kQTile;
+        mbar_arrive_expect_tx(bar(Lay::B_QF + s), 2 * Lay::QT);
+        for (int db = 0; db < D / 64; ++db) {
+          tma_load_3d(sb + Lay::Q + s * Lay::QT + db * 8192, &tmQ, bar(Lay::B_QF + s), db * 64, row, bh);
+          tma_load_3d(sb + Lay::DO + s * Lay::QT + db * 8192, &tmDO, bar(Lay::B_QF + s), db * 64, row, bh);
+        }
+        issued = it + 1;
+      }
+      if (!ok) {
+        mbar_wait_teardown(bar(Lay::B_KV), 0);
+        for (int it = issued >= kStages ? issued - kStages : 0; it < issued; ++it)
+          mbar_wait_teardown(bar(Lay::B_QF + it % kStages), (it / kStages) & 1);
+      }
     }
-    mbar_arrive_expect_tx(bar_qd, 2 * Lay::TILE);
-    for (int db = 0; db < D / 64; ++db) {
-      tma_load_3d(sb + Lay::Q + db * 16384, &tmQ, bar_qd, db * 64, kt * kTile, bh);
-      tma_load_3d(sb + Lay::DO + db * 16384, &tmDO, bar_qd, db * 64, kt * kTile, bh);
-    }
-  }
-
-  const int r = warp * 32 + lane;  // TMEM lane: key row of S^T/dP^T/dV/dK, feature of dQ^T
-  bool ok = true;
-  int issued_qd = 1;
-
-  for (int i = kt; i < ntiles && ok; ++i) {
-    const int it = i - kt;
-    {  // query-tile statistics into shared memory (rows beyond S contribute nothing)
-      const int q = i * kTile + r;
-      s_lse[r] = q < S ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
-      s_d[r] = q < S ? dvec[(int64_t)bh * S + q] : 0.f;
-    }
-    if (threadIdx.x == 0) {
-      const bool got = (it > 0 || mbar_wait(bar_kv, 0, &s_abort, status)) &&
-                       mbar_wait(bar_qd, it & 1, &s_abort, status);
-      if (got) {
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_f32acc(kFmtF16, 128, kQTile, 0, 0);   // K-major x K-major
+      constexpr uint32_t idesc_acc = idesc_f32acc(kFmtF16, 128, D, 0, 1);      // K-major x MN-major
+      constexpr uint32_t idesc_dq = idesc_f32acc(kFmtF16, 128, kQTile, 1, 1);  // MN-major x MN-major
+      bool ok = mbar_wait(bar(Lay::B_KV), 0, &s_abort, status);
+      auto products = [&](int jt) {  // dV, dK, dQ^T of sub-tile jt
+        const int b = jt & 1, s = jt % kStages;
+        if (!mbar_wait(bar(Lay::B_DSF + b), (jt >> 1) & 1, &s_abort, status)) return false;
         tc_fence_after();
+        const uint32_t sP = sb + Lay::P + b * Lay::PT, sDS = sb + Lay::DS + b * Lay::PT;
+        const uint32_t sQ = sb + Lay::Q + s * Lay::QT, sDO = sb + Lay::DO + s * Lay::QT;
+#pragma unroll
+        for (int kk = 0; kk < kQTile / 16; ++kk) {  // reduction over the 64 queries
+          const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
+          umma_ss(tDV, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sDO + kk * 2048, 8192, 1024), idesc_acc,
+                  acc);
+          umma_ss(tDK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc,
+                  acc);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kKTile / 16; ++kk)  // reduction over the 128 keys
+          umma_ss(tmem + 128 * b, sdesc_sw128(sb + Lay::K + kk * 2048, 16384, 1024),
+                  sdesc_sw128(sDS + kk * 2048, 8192, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+        umma_commit(bar(Lay::B_MM + b));
+        umma_commit(bar(Lay::B_QE + s));
+        return true;
+      };
+      for (int it = 0; it < nit && ok; ++it) {
+        const int b = it & 1, s = it % kStages;
+        ok = mbar_wait(bar(Lay::B_QF + s), (it / kStages) & 1, &s_abort, status);
+        // buffer pair b: its dQ^T of sub-tile it-2 has been read out of tensor memory
+        if (ok && it >= 2) ok = mbar_wait(bar(Lay::B_DQF + b), ((it >> 1) - 1) & 1, &s_abort, status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sQ = sb + Lay::Q + s * Lay::QT, sDO = sb + Lay::DO + s * Lay::QT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tS, sdesc_sw128(sb + Lay::K + koff, 16, 1024), sdesc_sw128(sb + Lay::Q + koff, 16, 1024),
-                       idesc_kk, kk > 0);
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32, qo = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_ss(tmem + 128 * b, sdesc_sw128(sb + Lay::K + ko, 16, 1024), sdesc_sw128(sQ + qo, 16, 1024), idesc_s,
+                  kk > 0 ? 1u : 0u);
+          umma_ss(tmem + 128 * b + 64, sdesc_sw128(sb + Lay::V + ko, 16, 1024), sdesc_sw128(sDO + qo, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
         }
+        umma_commit(bar(Lay::B_SF + b));
+        if (it >= 1) ok = products(it - 1);
+      }
+      if (ok && nit >= 1) ok = products(nit - 1);
+      umma_commit(bar(Lay::B_FIN));  // dV, dK final once every product above has completed
+      umma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_teardown(bar(Lay::B_DRAIN), 0);
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- compute: P^T and dS^T rows
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row inside the tile = TMEM lane
+    const int ct = threadIdx.x - 64;    // 0..127 inside the compute group
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int key = kt * kKTile + r;
+    float* s_lse = reinterpret_cast<float*>(smem + Lay::STAT);
+    float* s_d = s_lse + 2 * kQTile;
+    bool ok = true;
+    for (int it = 0; it < nit; ++it) {
+      const int b = it & 1, i = i0 + it;
+      // statistics of the sub-tile into buffer b (its previous readers, sub-tile it-2, are done: same threads)
+      if (ct < kQTile) {
+        const int q = i * kQTile + ct;
+        s_lse[b * kQTile + ct] = q < S ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
+        s_d[b * kQTile + ct] = q < S ? dvec[(int64_t)bh * S + q] : 0.f;
+      }
+      ok = named_barrier_and(kBarCompute, 128, ok);
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_abort, status));
+      float sv[64], dp[64];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + 128 * b + lane_base, *reinterpret_cast<float(*)[32]>(&sv[0]));
+        tmem_ld32(tmem + 128 * b + lane_base + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+        tmem_ld32(tmem + 128 * b + 64 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[0]));
+        tmem_ld32(tmem + 128 * b + 96 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[32]));
+        tmem_ld_wait();
+      }
+      uint32_t pk[32], dk[32];
+      float ds_max = 0.f;
+      if (ok) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tDP, sdesc_sw128(sb + Lay::V + koff, 16, 1024), sdesc_sw128(sb + Lay::DO + koff, 16, 1024),
-                       idesc_kk, kk > 0);
+        for (int c = 0; c < kQTile; c += 2) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int q = i * kQTile + c + e;
+            float pv = ex2(sv[c + e] * scale_log2 - s_lse[b * kQTile + c + e]);
+            if (q < key) pv = 0.f;  // query q does not see key `key`
+            p2[e] = pv;
+            d2[e] = pv * (dp[c + e] - s_d[b * kQTile + c + e]) * scale;
+            ds_max = fmaxf(ds_max, fabsf(d2[e]));
+          }
+          pk[c / 2] = pack_half2_rn(p2[0], p2[1]);
+          dk[c / 2] = pack_half2_rn(d2[0], d2[1]);
         }
-        umma_commit(bar_mm1);
-      } else {
-        s_abort = 1;
+        if (__any_sync(0xffffffffu, !(ds_max <= 65504.f)) && lane == 0) set_status(status, LH_ERR_RANGE);
+        // P/dS buffer b is free once the products of sub-tile it-2 have completed
+        if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_abort,
+                                                            status));
+      }
+      if (ok) {
+        uint8_t* sP = smem + Lay::P + b * Lay::PT;
+        uint8_t* sDS = smem + Lay::DS + b * Lay::PT;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunk ch holds queries 8 ch .. 8 ch + 7
+          const uint32_t off = sw128_offset(r, ch);
+          *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(sDS + off) = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_DSF + b));
       }
     }
-    ok = mbar_wait(bar_mm1, it & 1, &s_abort, status);
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-
-    // P^T and dS^T rows of key r
-    const bool diag = (i == kt);
-    uint8_t* sP = smem + Lay::P;
-    uint8_t* sDS = smem + Lay::DS;
-    float ds_max = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float sv[32], dp[32];
-      tmem_ld32(tS + lane_base + c * 32, sv);
-      tmem_ld32(tDP + lane_base + c * 32, dp);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        float p[8], ds[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int qc = c * 32 + q8 * 8 + e;  // query column inside the tile
-          float pv = ex2(sv[q8 * 8 + e] * scale_log2 - s_lse[qc]);
-          if (diag && qc < r) pv = 0.f;        // query qc does not see key r
-          p[e] = pv;
-          ds[e] = pv * (dp[q8 * 8 + e] - s_d[qc]) * scale;  // scaled by the head's dO_g scale
-          ds_max = fmaxf(ds_max, fabsf(ds[e]));
-        }
-        const int col = c * 32 + q8 * 8;
-        const uint32_t off = (col >> 6) * 16384 + sw128_offset(r, (col & 63) >> 3);
-        *reinterpret_cast<uint4*>(sP + off) =
-            make_uint4(pack_half2_rn(p[0], p[1]), pack_half2_rn(p[2], p[3]), pack_half2_rn(p[4], p[5]),
-                       pack_half2_rn(p[6], p[7]));
-        *reinterpret_cast<uint4*>(sDS + off) =
-            make_uint4(pack_half2_rn(ds[0], ds[1]), pack_half2_rn(ds[2], ds[3]), pack_half2_rn(ds[4], ds[5]),
-                       pack_half2_rn(ds[6], ds[7]));
-      }
-    }
-    if (__any_sync(0xffffffffu, !(ds_max <= 65504.f)) && lane == 0) set_status(status, LH_ERR_RANGE);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    // epilogue: dV and dK rows of this key tile (the products' accumulators are final after B_FIN)
+    ok = named_barrier_and(kBarCompute, 128, ok);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FIN), 0, &s_abort, status));
+    if (ok) {
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {  // reduction over the 128 query rows
-        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        umma_ss(tDV, sdesc_sw128(sb + Lay::P + aoff, 16, 1024), sdesc_sw128(sb + Lay::DO + kk * 2048, 16384, 1024),
-                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-        umma_ss(tDK, sdesc_sw128(sb + Lay::DS + aoff, 16, 1024), sdesc_sw128(sb + Lay::Q + kk * 2048, 16384, 1024),
-                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-      }
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tacc = which == 0 ? tDV : tDK;
+        float* dst_base = which == 0 ? dvg : dkg;
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {  // reduction over the 128 key rows
-        umma_ss(tS, sdesc_sw128(sb + Lay::K + kk * 2048, 16384, 1024),
-                     sdesc_sw128(sb + Lay::DS + kk * 2048, 16384, 1024), idesc_dq, kk > 0);
-      }
-      umma_commit(bar_mm2);
-    }
-    ok = mbar_wait(bar_mm2, it & 1, &s_abort, status);
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    if (threadIdx.x == 0 && i + 1 < ntiles) {  // Q_i and dO_i are no longer read
-      mbar_arrive_expect_tx(bar_qd, 2 * Lay::TILE);
-      for (int db = 0; db < D / 64; ++db) {
-        tma_load_3d(sb + Lay::Q + db * 16384, &tmQ, bar_qd, db * 64, (i + 1) * kTile, bh);
-        tma_load_3d(sb + Lay::DO + db * 16384, &tmDO, bar_qd, db * 64, (i + 1) * kTile, bh);
-      }
-      issued_qd = it + 2;
-    }
-    // dQ^T: lane r = feature r, columns = the 128 query rows of tile i
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tacc + lane_base + c * 32, v);
+          tmem_ld_wait();
+          if (key < S) {
+            float4* dst = reinterpret_cast<float4*>(dst_base + ((int64_t)bh * S + key) * D + c * 32);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      tmem_ld32(tS + lane_base + c * 32, v);
-      tmem_ld_wait();
-      if (r < D) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = i * kTile + c * 32 + e;
-          if (q < S) atomicAdd(dqacc + ((int64_t)bh * S + q) * D + r, v[e] * inv_scale);
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
+                                    v[q4 * 4 + 3] * inv_scale);
+          }
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();  // S^T columns, P and dS tiles and the statistics are reused by the next query tile
-    tc_fence_after();
+  } else {
+    // ---------------------------------------------------------------- drain: dQ^T -> shared tile -> TMA reduce-add
+    const int quarter = warp & 3;
+    const int f = quarter * 32 + lane;  // feature = TMEM lane of dQ^T
+    const int dt = threadIdx.x - 192;   // 0..127 inside the drain group
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + Lay::DQ);
+    bool ok = true;
+    for (int it = 0; it < nit; ++it) {
+      const int b = it & 1, i = i0 + it;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(Lay::B_MM + b), (it >> 1) & 1, &s_abort, status));
+      float v[64];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + 128 * b + lane_base, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(tmem + 128 * b + lane_base + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_DQF + b));  // TMEM pair b may take the next S^T
+      }
+      // the previous reduce must have finished reading the staging tile before it is overwritten
+      if (dt == 0) bulk_wait_group_read0();
+      ok = named_barrier_and(kBarDrain, 128, ok);
+      if (!ok) break;
+      if (f < D) {
+        float* col = stage + (f >> 5) * (kQTile * 32) + (f & 31);  // box (f/32): [64 q][32 f]
+#pragma unroll
+        for (int c = 0; c < kQTile; ++c) col[c * 32] = v[c] * inv_scale;
+      }
+      fence_proxy_async_smem();
+      named_barrier_and(kBarDrain, 128, true);
+      if (dt == 0) {
+        for (int fb = 0; fb < D / 32; ++fb)
+          tma_reduce_add_3d(&tmDQ, smem_u32(stage + fb * kQTile * 32), fb * 32, i * kQTile, bh);
+        bulk_commit_group();
+      }
+    }
+    if (dt == 0) bulk_wait_group0();  // every reduction has landed before the block exits
   }
 
-  if (ok) {
-    const int krow = kt * kTile + r;
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t tacc = which == 0 ? tDV : tDK;
-      float* dst_base = which == 0 ? dvg : dkg;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float v[32];
-        tmem_ld32(tacc + lane_base + c * 32, v);
-        tmem_ld_wait();
-        if (krow < S) {
-          float4* dst = reinterpret_cast<float4*>(dst_base + ((int64_t)bh * S + krow) * D + c * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
-                                  v[q4 * 4 + 3] * inv_scale);
-        }
-      }
-    }
-  } else if (threadIdx.x == 0) {
-    umma_commit(bar_drain);
-    mbar_wait_teardown(bar_drain, 0);
-    mbar_wait_teardown(bar_kv, 0);
-    mbar_wait_teardown(bar_qd, (issued_qd - 1) & 1);
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -273,17 +332,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 int launch_bwd_t(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse, const float* dvec,
                  const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mdo;
-  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH) ||
-      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH))
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH, kQTile) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH, kKTile) ||
+      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH, kKTile) || make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH, kQTile) ||
+      make_tmap_f32_3d(&mdq, dqacc, D, dm.S, dm.BH, 32, kQTile))
     return LH_ERR_CUDA;
   const int smem = BwdLayout<D>::BYTES + 1024;
   if (cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LH_ERR_CUDA;
-  const int nt = (dm.S + kTile - 1) / kTile;
+  const int nt = (dm.S + kKTile - 1) / kKTile;
   KernelTimer timer("attn_bwd", st);
-  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, lse, dvec, dinv, dqacc, dkg, dvg,
-                                                               dm.S, nt, 1.0f / sqrtf((float)D), dm.status);
+  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, dvec, dinv, dkg, dvg, dm.S,
+                                                               1.0f / sqrtf((float)D), dm.status);
   return check_launch();
 }
 

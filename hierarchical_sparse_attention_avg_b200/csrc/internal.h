@@ -62,8 +62,10 @@ int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* 
                     const float* dvec, const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm,
                     cudaStream_t st);
 
-// Encode a 3-D fp16 tensor map over [BH][rows][d] with a {64, 128, 1} box and 128-byte swizzle.
-int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh);
+// Encode a 3-D fp16 tensor map over [BH][rows][d] with a {64, box_rows, 1} box and 128-byte swizzle.
+int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_rows = 128);
+// Encode a 3-D fp32 tensor map over [BH][rows][d] with a {box_cols, box_rows, 1} box, no swizzle.
+int make_tmap_f32_3d(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_cols, int box_rows);
 
 inline int check_launch() { return cudaGetLastError() == cudaSuccess ? LH_OK : LH_ERR_CUDA; }
 
