@@ -67,7 +67,7 @@ int make_dims(const lh_params* P, LhDims* dm) {
   // what the kernels are built for
   if (P->d != 64 && P->d != 128) return LH_ERR_UNSUPPORTED;
   if (P->p != 2 && P->p != 4 && P->p != 8) return LH_ERR_UNSUPPORTED;
-  if (P->L > 5 || w > 512) return LH_ERR_UNSUPPORTED;
+  if (P->L > kMaxL || w > 512) return LH_ERR_UNSUPPORTED;
   if (nPartial > 0 && P->k / P->C > 512) return LH_ERR_UNSUPPORTED;
   if (BH > 65535 || R > INT32_MAX / 2) return LH_ERR_UNSUPPORTED;
   return LH_OK;

@@ -15,6 +15,9 @@
 
 namespace lh {
 
+// Largest level count the kernels are built for (the entry points reject more); loops over levels unroll to it.
+constexpr int kMaxL = 5;
+
 // ------------------------------------------------------------------------------------------------------------
 // Sizes of one call, computed on the host and passed by value.
 // ------------------------------------------------------------------------------------------------------------
@@ -125,6 +128,17 @@ __device__ __forceinline__ void st_stream16(void* p, const uint4& v) {
 // ------------------------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only); copies are grouped per thread by commit, and a wait
+// returns once at most N of this thread's most recent groups are still pending.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

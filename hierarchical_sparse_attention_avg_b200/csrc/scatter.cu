@@ -68,92 +68,281 @@ __device__ __forceinline__ float head_scale(float amax) {
   return ldexpf(1.f, 10 - e);
 }
 
-// Tokens per row group in the token-major kernels: every slot lookup of the group is issued before any row load,
-// so a thread keeps up to kMaxL * kTok independent loads in flight instead of a chain of dependent ones.
-constexpr int kTok = 4;
-constexpr int kMaxL = 5;
+// Window sums for the scatter-back (offset, one tensor) and the unpool backward (three tensors).
+//
+// A tile is T consecutive "keys" of one head, key0 a multiple of T; key = t + 1 for the scatter (entry
+// j = key/w - 1) and key = t for the unpool (j = key/w).  Windows are powers of two, so a level with w <= T has
+// T/w entries in the tile and a wider level exactly one.  Per tile:
+//   1. every thread holds at most kH slots of the tile's entry list (loaded one tile ahead); a block-wide
+//      ballot scan numbers the selected entries (compact index) and lists their source rows;
+//   2. each warp copies the selected rows of its own entries, every tensor, to shared memory with cp.async (the
+//      first M rows of the tile; rows beyond M, which only very dense selections reach, are read from global
+//      memory where they are used), and marks the keys that a selected "fine" entry covers in a bitmap;
+//   3. a row group (d/8 lanes) owns PP consecutive keys.  Levels with w >= PP ("uniform") have one entry for the
+//      whole group: their rows are summed once into a base row, rounded, packed and stored to every key.  Levels
+//      with w < PP ("fine") differ per key: each key marked in the bitmap is then recomputed as base + its fine
+//      rows (fp32, one rounding) and stored again over the base value.  Weights are 1 (scatter) and
+//      2^-level-shift (unpool, exact).
+// The loop is software-pipelined over the block's tiles: while tile i is summed and stored, the rows of tile
+// i+1 are in flight to the other shared-memory stage and the slots of tile i+2 to registers, so no tile waits
+// for a full memory round trip.
+constexpr int kWinThreads = 256;
+constexpr int kWinWarps = kWinThreads / 32;
+constexpr int kWinStageBytes = 24 * 1024;  // staged rows per stage, all tensors
 
-// Row group g covers the kTok tokens whose "key" is g*kTok .. g*kTok + kTok - 1, where key = t + 1 for the offset
-// scatter (entry j = key/w - 1) and key = t for the unpool (j = key/w).  Windows are powers of two, so for every
-// level with w >= kTok the whole group reads ONE entry (one slot lookup, one row load, added to all kTok tokens);
-// only narrower levels need per-token lookups.  Rows are summed in fp32 with per-level weights.
-template <int D, bool kOffset>
-__device__ __forceinline__ void token_sum(const float* __restrict__ src, const int32_t* __restrict__ sl, int bh,
-                                          int key0, int lane, const LhDims& dm, float (&acc)[kTok][8]) {
-  int s[kMaxL][kTok];
+template <int D, int P, int NT>
+struct WinCfg {
+  static constexpr int G = D / 8;                  // lanes per row
+  static constexpr int RG = kWinThreads / G;       // row groups
+  static constexpr int PP = (NT == 1 && D == 128) ? 16 : 8;  // keys per row group
+  static constexpr int T = RG * PP;                // keys per tile
+  static constexpr int M = kWinStageBytes / (NT * D * 4);
+  static constexpr int LP = P == 2 ? 1 : (P == 4 ? 2 : 3);  // log2 p
+  // entries of level l in a tile, and the first entry of level l in the tile's list
+  __host__ __device__ static constexpr int n_ent(int l) { return (1 << (l * LP)) <= T ? T >> (l * LP) : 1; }
+  __host__ __device__ static constexpr int ent_base(int l) { return l == 0 ? 0 : ent_base(l - 1) + n_ent(l - 1); }
+  static constexpr int kMaxEnt = ent_base(kMaxL);
+  static constexpr int kH = (kMaxEnt + kWinThreads - 1) / kWinThreads;  // entries per thread
+  static constexpr int kWords = T / 32;                                  // fine-key bitmap words
+  __host__ __device__ static constexpr bool uniform(int l) { return (1 << (l * LP)) >= PP; }
+  __host__ __device__ static constexpr float weight(int l, bool offset) {
+    return offset ? 1.0f : 1.0f / (float)(1 << (l * LP));  // exact: a power of two
+  }
+  static_assert(T % 32 == 0 && PP <= 32 && 32 % PP == 0, "row groups tile the bitmap words");
+};
+
+// The tile-independent part of one of a thread's entries: level (-1 beyond the last level), shift, offset in
+// the level's run within the tile, entry offset including the scatter's -1, level size, slot-row offset, and
+// whether the level is fine.
+struct WinEntry {
+  int lev, sh, r, e, nl, off;
+  bool fine;
+};
+
+template <int D, int P, int NT, bool kOffset>
+__device__ __forceinline__ WinEntry win_entry(int i, const LhDims& dm) {
+  using C = WinCfg<D, P, NT>;
+  WinEntry w{-1, 0, 0, 0, 0, 0, false};
 #pragma unroll
-  for (int lev = 0; lev < kMaxL; ++lev) {
-#pragma unroll
-    for (int u = 0; u < kTok; ++u) s[lev][u] = -1;
-    if (lev >= dm.L) continue;
-    const int sh = dm.wlog[lev];
-    if ((1 << sh) >= kTok) {
-      const int j = (key0 >> sh) - (kOffset ? 1 : 0);
-      if (j >= 0 && j < dm.Nl[lev]) s[lev][0] = sl[dm.off[lev] + j];
-    } else {
-#pragma unroll
-      for (int u = 0; u < kTok; ++u) {
-        const int j = ((key0 + u) >> sh) - (kOffset ? 1 : 0);
-        if (j >= 0 && j < dm.Nl[lev]) s[lev][u] = sl[dm.off[lev] + j];
-      }
+  for (int l = 0; l < kMaxL; ++l) {
+    if (l < dm.L && i >= C::ent_base(l) && i < C::ent_base(l) + C::n_ent(l)) {
+      w.lev = l;
+      w.sh = l * C::LP;
+      w.r = i - C::ent_base(l);
+      w.e = w.r - (kOffset ? 1 : 0);
+      w.nl = dm.Nl[l];
+      w.off = dm.off[l];
+      w.fine = !C::uniform(l);
     }
   }
+  return w;
+}
+
+// Slot of entry `w` in the tile of head bh starting at key0 (-1: not selected, or outside the level).
+__device__ __forceinline__ int win_slot(const WinEntry& w, int bh, int key0, const int32_t* __restrict__ slot,
+                                        const LhDims& dm) {
+  const int j = (key0 >> w.sh) + w.e;
+  return (w.lev >= 0 && j >= 0 && j < w.nl) ? slot[(int64_t)bh * dm.R + w.off + j] : -1;
+}
+
+// Numbers the selected entries of a tile (compact index into s_cidx, source row into s_src), starts the copy of
+// the first M selected rows of every tensor into stage buffer `buf`, clears the stage's fine-key bitmap and
+// returns in (fw, fm) the bitmap word and bits of each selected fine entry of this thread (fm = 0: none), to be
+// set once the clearing is visible to every thread.
+template <int D, int P, int NT>
+__device__ __forceinline__ void win_stage(const int (&s)[WinCfg<D, P, NT>::kH],
+                                          const WinEntry (&we)[WinCfg<D, P, NT>::kH], int bh,
+                                          const float* const (&src)[3], const LhDims& dm, int* s_cidx, int* s_src,
+                                          int* s_wcount, unsigned* s_fine, float* buf,
+                                          int (&fw)[WinCfg<D, P, NT>::kH], unsigned (&fm)[WinCfg<D, P, NT>::kH]) {
+  using C = WinCfg<D, P, NT>;
+  constexpr int kH = C::kH;
+  const int tid = threadIdx.x, wid = tid >> 5, wl = tid & 31;
+  unsigned m[kH];
 #pragma unroll
-  for (int u = 0; u < kTok; ++u)
+  for (int h = 0; h < kH; ++h) {
+    m[h] = __ballot_sync(0xffffffffu, s[h] >= 0);
+    if (wl == 0) s_wcount[h * kWinWarps + wid] = __popc(m[h]);
+    // a fine entry at run offset r covers tile keys r*w .. r*w + w - 1 (w < PP <= 32: one bitmap word)
+    const int k0 = we[h].r << we[h].sh;
+    fw[h] = k0 >> 5;
+    fm[h] = (s[h] >= 0 && we[h].fine) ? ((2u << ((1 << we[h].sh) - 1)) - 1u) << (k0 & 31) : 0u;
+  }
+  __syncthreads();
+  if (tid < C::kWords) s_fine[tid] = 0u;
+  int c[kH];
+  int run = 0;  // selected entries of the earlier groups
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+  for (int h = 0; h < kH; ++h) {
+    const int4 lo = *reinterpret_cast<const int4*>(s_wcount + h * kWinWarps);
+    const int4 hi = *reinterpret_cast<const int4*>(s_wcount + h * kWinWarps + 4);
+    const int w8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    int pre = 0, tot = 0;
 #pragma unroll
-  for (int lev = 0; lev < kMaxL; ++lev) {
-    if (lev >= dm.L) continue;
-    const int sh = dm.wlog[lev];
-    const float wgt = kOffset ? 1.0f : __uint_as_float((127u - (uint32_t)sh) << 23);  // 2^-sh, exact
-    if ((1 << sh) >= kTok) {
-      if (s[lev][0] >= 0) {
-        float f[8];
-        load8f(src + ((int64_t)bh * dm.S + s[lev][0]) * D + lane * 8, f);
+    for (int w = 0; w < kWinWarps; ++w) {
+      pre += w < wid ? w8[w] : 0;
+      tot += w8[w];
+    }
+    c[h] = s[h] >= 0 ? run + pre + __popc(m[h] & ((1u << wl) - 1u)) : -1;
+    run += tot;
+    const int i = tid + h * kWinThreads;
+    if (i < C::kMaxEnt) s_cidx[i] = c[h];
+    if (c[h] >= 0) s_src[c[h]] = s[h];
+  }
+  // the warp copies the rows of its own selected entries: lane x moves 16-byte chunks x, x + 32, ...
+  constexpr int kChunks = D / 4;  // 16-byte chunks per fp32 row
 #pragma unroll
-        for (int u = 0; u < kTok; ++u)
+  for (int h = 0; h < kH; ++h) {
+    unsigned mm = m[h];
+    while (mm) {
+      const int src_lane = __ffs(mm) - 1;
+      mm &= mm - 1;
+      const int cc = __shfl_sync(0xffffffffu, c[h], src_lane);
+      const int row = __shfl_sync(0xffffffffu, s[h], src_lane);
+      if (cc < C::M) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(f[i], wgt, acc[u][i]);
-      }
-    } else {
+        for (int t = 0; t < NT; ++t) {
+          const float* g = src[t] + ((int64_t)bh * dm.S + row) * D;
+          float* sb = buf + (t * C::M + cc) * D;
 #pragma unroll
-      for (int u = 0; u < kTok; ++u) {
-        if (s[lev][u] >= 0) {
-          float f[8];
-          load8f(src + ((int64_t)bh * dm.S + s[lev][u]) * D + lane * 8, f);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(f[i], wgt, acc[u][i]);
+          for (int x = wl; x < kChunks; x += 32) cp_async16(smem_u32(sb + x * 4), g + x * 4);
         }
       }
     }
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) scatter_kernel(const float* __restrict__ og, const int32_t* __restrict__ slot,
-                                                      __nv_bfloat16* __restrict__ o, LhDims dm) {
-  constexpr int G = D / 8;
-  const int lane = threadIdx.x % G;
-  const int gph = (dm.N + kTok) / kTok;  // row groups per head: keys t + 1 = 1 .. N
-  const int64_t ngrp = (int64_t)dm.BH * gph;
-  // grid-stride over row groups: a few resident blocks per SM instead of one short-lived block per 64 tokens
-  for (int64_t grp = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G; grp < ngrp;
-       grp += (int64_t)gridDim.x * (256 / G)) {
-    const int bh = (int)(grp / gph);
-    const int key0 = (int)(grp % gph) * kTok;
-    float acc[kTok][8];
-    token_sum<D, true>(og, slot + (int64_t)bh * dm.R, bh, key0, lane, dm, acc);
+template <int kH>
+__device__ __forceinline__ void win_mark(const int (&fw)[kH], const unsigned (&fm)[kH], unsigned* s_fine) {
 #pragma unroll
-    for (int u = 0; u < kTok; ++u) {
-      const int t = key0 + u - 1;
-      if (t >= 0 && t < dm.N) st_stream16(o + ((int64_t)bh * dm.N + t) * D + lane * 8, pack8_rn(acc[u]));
-    }
-  }
+  for (int h = 0; h < kH; ++h)
+    if (fm[h]) atomicOr(s_fine + fw[h], fm[h]);
 }
 
-// One group per gathered row: dog[s] = fp32 window sum of dout.  With amax non-null, also the running per-head
-// maximum magnitude (non-negative fp32 bit patterns order like their values).
+template <int D, int P, bool kOffset, int NT>
+__global__ void __launch_bounds__(kWinThreads, 4) window_sum_kernel(const float* __restrict__ src0,
+                                                                   const float* __restrict__ src1,
+                                                                   const float* __restrict__ src2,
+                                                                   const int32_t* __restrict__ slot,
+                                                                   __nv_bfloat16* dst0, __nv_bfloat16* dst1,
+                                                                   __nv_bfloat16* dst2, LhDims dm) {
+  using C = WinCfg<D, P, NT>;
+  constexpr int G = C::G, PP = C::PP, T = C::T, M = C::M, LP = C::LP, kH = C::kH;
+  extern __shared__ __align__(16) float s_buf[];  // [2 stages][NT][M][D]
+  __shared__ int s_cidx[2][C::kMaxEnt];
+  __shared__ int s_src[2][C::kMaxEnt];
+  __shared__ __align__(16) int s_wcount[2][kH * kWinWarps];
+  __shared__ unsigned s_fine[2][C::kWords];
+  const float* const src[3] = {src0, src1, src2};
+  __nv_bfloat16* const dst[3] = {dst0, dst1, dst2};
+  const int tid = threadIdx.x, lane = tid % G, x0 = (tid / G) * PP;
+  // Tiles are numbered head-major (tile = bh * tph + kt) and visited with stride gridDim.x; (bh, kt) is advanced
+  // incrementally.  Three tiles are live: the one summed (0), the one staged (1) and the one whose slots load (2).
+  const int tph = (dm.N + (kOffset ? 1 : 0) + T - 1) / T;  // tiles per head
+  const int sq = (int)(gridDim.x / (unsigned)tph), sr = (int)(gridDim.x % (unsigned)tph);
+  int bh0 = (int)(blockIdx.x / (unsigned)tph), kt0 = (int)(blockIdx.x % (unsigned)tph);
+  if (bh0 >= dm.BH) return;
+  int bh1 = bh0 + sq, kt1 = kt0 + sr;
+  if (kt1 >= tph) { kt1 -= tph; ++bh1; }
+  int bh2 = bh1 + sq, kt2 = kt1 + sr;
+  if (kt2 >= tph) { kt2 -= tph; ++bh2; }
+  WinEntry we[kH];
+#pragma unroll
+  for (int h = 0; h < kH; ++h) we[h] = win_entry<D, P, NT, kOffset>(tid + h * kWinThreads, dm);
+  int sl[kH], fw[kH];
+  unsigned fm[kH];
+#pragma unroll
+  for (int h = 0; h < kH; ++h) sl[h] = win_slot(we[h], bh0, kt0 * T, slot, dm);
+  win_stage<D, P, NT>(sl, we, bh0, src, dm, s_cidx[0], s_src[0], s_wcount[0], s_fine[0], s_buf, fw, fm);
+  cp_async_commit();
+  if (bh1 < dm.BH)
+#pragma unroll
+    for (int h = 0; h < kH; ++h) sl[h] = win_slot(we[h], bh1, kt1 * T, slot, dm);
+  __syncthreads();
+  win_mark<kH>(fw, fm, s_fine[0]);
+  for (int it = 0; bh0 < dm.BH; ++it) {
+    const int b = it & 1;
+    const bool has1 = bh1 < dm.BH;  // block-uniform
+    if (has1)
+      win_stage<D, P, NT>(sl, we, bh1, src, dm, s_cidx[b ^ 1], s_src[b ^ 1], s_wcount[b ^ 1], s_fine[b ^ 1],
+                          s_buf + (b ^ 1) * NT * M * D, fw, fm);
+    cp_async_commit();
+    if (bh2 < dm.BH)
+#pragma unroll
+      for (int h = 0; h < kH; ++h) sl[h] = win_slot(we[h], bh2, kt2 * T, slot, dm);
+    cp_async_wait<1>();  // this thread's copies for the summed tile are done ...
+    __syncthreads();     // ... and everyone's are visible, as is the cleared bitmap of the staged tile
+    if (has1) win_mark<kH>(fw, fm, s_fine[b ^ 1]);
+    const int bh = bh0, key0 = kt0 * T;
+    const int* ci = s_cidx[b];
+    const int* cs = s_src[b];
+    const float* sb = s_buf + b * NT * M * D;
+    const int64_t gbase = (int64_t)bh * dm.S * D + lane * 8;  // row 0 of this head in the sources
+    // the source row of compact index c (staged copy when c < M), at this thread's 8 features
+    auto row_ptr = [&](int t, int c) -> const float* {
+      return c < M ? sb + (t * M + c) * D + lane * 8 : src[t] + gbase + (int64_t)cs[c] * D;
+    };
+    const unsigned fine = (s_fine[b][x0 >> 5] >> (x0 & 31)) & (PP == 32 ? ~0u : (1u << PP) - 1u);
+    const int tok0 = key0 + x0 - (kOffset ? 1 : 0);  // token of this row group's first key
+    const int64_t obase = ((int64_t)bh * dm.N + tok0) * D + lane * 8;
+    const bool whole = tok0 >= 0 && tok0 + PP <= dm.N;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float base[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int l = 0; l < kMaxL; ++l) {
+        if (C::uniform(l) && l < dm.L) {
+          const int c = ci[C::ent_base(l) + ((1 << (l * LP)) <= T ? x0 >> (l * LP) : 0)];
+          if (c >= 0) {
+            float f[8];
+            load8f(row_ptr(t, c), f);
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8) base[e8] = fmaf(f[e8], C::weight(l, kOffset), base[e8]);
+          }
+        }
+      }
+      const uint4 packed = pack8_rn(base);
+      __nv_bfloat16* out = dst[t] + obase;
+      if (whole) {
+#pragma unroll
+        for (int q = 0; q < PP; ++q) st_stream16(out + q * D, packed);
+      } else {
+#pragma unroll
+        for (int q = 0; q < PP; ++q)
+          if (tok0 + q >= 0 && tok0 + q < dm.N) st_stream16(out + q * D, packed);
+      }
+      // keys with a selected fine entry: base + fine rows, stored over the base value (same thread, same address)
+      unsigned f = fine;
+      while (f) {
+        const int q = __ffs(f) - 1;
+        f &= f - 1u;
+        if (tok0 + q < 0 || tok0 + q >= dm.N) continue;
+        float acc[8];
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) acc[e8] = base[e8];
+#pragma unroll
+        for (int l = 0; l < kMaxL; ++l) {
+          if (!C::uniform(l) && l < dm.L) {
+            const int c = ci[C::ent_base(l) + ((x0 + q) >> (l * LP))];
+            if (c >= 0) {
+              float fr[8];
+              load8f(row_ptr(t, c), fr);
+#pragma unroll
+              for (int e8 = 0; e8 < 8; ++e8) acc[e8] = fmaf(fr[e8], C::weight(l, kOffset), acc[e8]);
+            }
+          }
+        }
+        st_stream16(out + q * D, pack8_rn(acc));
+      }
+    }
+    bh0 = bh1; kt0 = kt1;
+    bh1 = bh2; kt1 = kt2;
+    bh2 += sq; kt2 += sr;
+    if (kt2 >= tph) { kt2 -= tph; ++bh2; }
+  }
+  cp_async_wait<0>();
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) scatter_bwd_kernel(const __nv_bfloat16* __restrict__ dout,
                                                           const int32_t* __restrict__ idx_g, float* __restrict__ dog,
@@ -258,64 +447,50 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__
   }
 }
 
-// blockIdx.y selects the tensor: 0 = dQ, 1 = dK, 2 = dV (fp32 gathered gradients).
-template <int D>
-__global__ void __launch_bounds__(256) unpool_bwd_kernel(const float* __restrict__ dqg, const float* __restrict__ dkg,
-                                                         const float* __restrict__ dvg, const int32_t* __restrict__ slot,
-                                                         __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
-                                                         LhDims dm) {
-  constexpr int G = D / 8;
-  const int which = blockIdx.y;
-  const int lane = threadIdx.x % G;
-  const int gph = (dm.N + kTok - 1) / kTok;
-  const int64_t ngrp = (int64_t)dm.BH * gph;
-  const float* src = which == 0 ? dqg : (which == 1 ? dkg : dvg);
-  __nv_bfloat16* out = which == 0 ? dq : (which == 1 ? dk : dv);
-  for (int64_t grp = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G; grp < ngrp;
-       grp += (int64_t)gridDim.x * (256 / G)) {
-    const int bh = (int)(grp / gph);
-    const int t0 = (int)(grp % gph) * kTok;  // key = t
-    float acc[kTok][8];
-    token_sum<D, false>(src, slot + (int64_t)bh * dm.R, bh, t0, lane, dm, acc);
-#pragma unroll
-    for (int u = 0; u < kTok; ++u)
-      if (t0 + u < dm.N) st_stream16(out + ((int64_t)bh * dm.N + t0 + u) * D + lane * 8, pack8_rn(acc[u]));
-  }
-}
 
 template <int D>
 int blocks_for(int64_t rows) {
   return (int)((rows + 256 / (D / 8) - 1) / (256 / (D / 8)));
 }
 
-// Blocks for a grid-stride kernel: enough for every row group, capped at what the device keeps resident at once
-// (blocks per SM from the occupancy calculator times the SM count), so the loop has no ragged last wave.
-template <typename Kernel>
-int resident_blocks(Kernel kernel, int64_t need) {
+// Launch a window_sum_kernel with a grid of at most the blocks the device keeps resident at once (occupancy
+// times the SM count): each block pipelines over many tiles.
+template <int D, int P, bool kOffset, int NT>
+int launch_window_sum(const float* s0, const float* s1, const float* s2, const int32_t* slot, __nv_bfloat16* d0,
+                      __nv_bfloat16* d1, __nv_bfloat16* d2, const LhDims& dm, cudaStream_t st) {
+  using C = WinCfg<D, P, NT>;
+  auto kernel = window_sum_kernel<D, P, kOffset, NT>;
+  const int smem = 2 * NT * C::M * D * (int)sizeof(float);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return LH_ERR_CUDA;
+  const int64_t tiles = (int64_t)dm.BH * ((dm.N + (kOffset ? 1 : 0) + C::T - 1) / C::T);
+  if (tiles >= (int64_t)1 << 31) return LH_ERR_UNSUPPORTED;
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWinThreads, smem);
   const int64_t cap = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
-  return (int)(need < cap ? need : cap);
+  const int grid = (int)(tiles < cap ? tiles : cap);
+  kernel<<<grid, kWinThreads, smem, st>>>(s0, s1, s2, slot, d0, d1, d2, dm);
+  return check_launch();
 }
 
-// `slices` launches share the device (gridDim.y), so each gets 1/slices of the resident blocks.
-template <int D, typename Kernel>
-int token_blocks(Kernel kernel, const LhDims& dm, int slices) {
-  const int b = resident_blocks(kernel, blocks_for<D>((int64_t)dm.BH * ((dm.N + kTok - 1) / kTok))) / slices;
-  return b > 0 ? b : 1;
+template <bool kOffset, int NT>
+int window_sum(const float* s0, const float* s1, const float* s2, const int32_t* slot, void* d0, void* d1, void* d2,
+               const LhDims& dm, cudaStream_t st) {
+  __nv_bfloat16 *o0 = (__nv_bfloat16*)d0, *o1 = (__nv_bfloat16*)d1, *o2 = (__nv_bfloat16*)d2;
+#define LH_WIN(DD, PPV) \
+  if (dm.d == DD && dm.p == PPV) return launch_window_sum<DD, PPV, kOffset, NT>(s0, s1, s2, slot, o0, o1, o2, dm, st);
+  LH_WIN(64, 2) LH_WIN(64, 4) LH_WIN(64, 8) LH_WIN(128, 2) LH_WIN(128, 4) LH_WIN(128, 8)
+#undef LH_WIN
+  return LH_ERR_UNSUPPORTED;
 }
 
 }  // namespace
 
 int launch_scatter(const float* og, const int32_t* slot, void* o, const LhDims& dm, cudaStream_t st) {
   KernelTimer timer("scatter", st);
-  if (dm.d == 64)
-    scatter_kernel<64><<<token_blocks<64>(scatter_kernel<64>, dm, 1), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
-  else
-    scatter_kernel<128><<<token_blocks<128>(scatter_kernel<128>, dm, 1), 256, 0, st>>>(og, slot, (__nv_bfloat16*)o, dm);
-  return check_launch();
+  return window_sum<true, 1>(og, og, og, slot, o, o, o, dm, st);
 }
 
 int launch_scatter_bwd(const void* dout, const int32_t* idx_g, float* dog, unsigned int* amax, const LhDims& dm,
@@ -353,13 +528,7 @@ int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax,
 int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st) {
   KernelTimer timer("unpool_bwd", st);
-  if (dm.d == 64)
-    unpool_bwd_kernel<64><<<dim3(token_blocks<64>(unpool_bwd_kernel<64>, dm, 3), 3), 256, 0, st>>>(
-        dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
-  else
-    unpool_bwd_kernel<128><<<dim3(token_blocks<128>(unpool_bwd_kernel<128>, dm, 3), 3), 256, 0, st>>>(
-        dqg, dkg, dvg, slot, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, dm);
-  return check_launch();
+  return window_sum<false, 3>(dqg, dkg, dvg, slot, dq, dk, dv, dm, st);
 }
 
 }  // namespace lh
