@@ -18,6 +18,9 @@ namespace lh {
 namespace {
 
 constexpr int kPoolThreads = 256;
+constexpr int kPoolStages = 3;  // batches of raw rows in flight per thread (cp.async into private shared slots)
+
+__host__ __device__ constexpr int pool_batch(int W) { return W < 8 ? W : 8; }
 
 __host__ __device__ constexpr int ipow(int b, int e) { return e == 0 ? 1 : b * ipow(b, e - 1); }
 
@@ -50,15 +53,52 @@ __device__ __forceinline__ uint4 round_pooled(const double (&sum)[8], double inv
   return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
 }
 
-// One group processes one block of W = P^(L-1) consecutive tokens of one head (one coarsest entry), building
-// every level of the pyramid inside the block in registers.
-template <int D, int P, int L>
+// Level-1 sums in fp32.  A level-1 entry sums p bf16 values; the sum is carried twice in fp32, rounded toward
+// +inf and toward -inf (IEEE directed rounding, subnormals kept).  The two chains bracket the exact value and stay
+// apart once any step rounded, so they are equal exactly when every step was exact -- the common case for p bf16
+// values -- and an exact fp32 sum is also what the fp64 order of the definition produces.  Then the pooled value
+// bf16_RN(sum / p) is the bf16 rounding of the fp32 value sum * 2^-log2(p) (exact while that is a normal number)
+// and the fp64 sum for the levels above is one widening per entry instead of one per element.  A lane whose
+// chains differ recomputes the entry in fp64 from the raw values.
+__device__ __forceinline__ float add_up(float a, float b) {
+  float r;
+  asm("add.rp.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float add_dn(float a, float b) {
+  float r;
+  asm("add.rm.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float mul_rn(float a, float b) {  // no flush of subnormal results
+  float r;
+  asm("mul.rn.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+// Upper and lower chain agree: same bits, or both zero (an exact zero sum is +0 upward and -0 downward).
+__device__ __forceinline__ bool same_sum(float up, float dn) {
+  const uint32_t a = __float_as_uint(up), b = __float_as_uint(dn);
+  return a == b || ((a | b) & 0x7FFFFFFFu) == 0u;
+}
+// Zero or a normal, finite number (tested on the bits, independent of flush-to-zero).
+__device__ __forceinline__ bool zero_or_normal(float x) {
+  const uint32_t e = (__float_as_uint(x) >> 23) & 0xFFu;
+  return (__float_as_uint(x) & 0x7FFFFFFFu) == 0u || (e != 0u && e != 0xFFu);
+}
+
+// One group builds every level of the pyramid over one block of W = P^(L-1) consecutive tokens of one head (one
+// coarsest entry): level 1 as above, levels >= 2 in fp64 registers, in the order the definition fixes.  The raw
+// rows stream through kPoolStages batches of TB rows per thread, copied with cp.async into shared-memory slots
+// private to the thread (so no block barrier is needed) while earlier batches are summed.
+template <int D, int P, int L, bool kScore>
 __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, LhDims dm) {
   constexpr int G = D / 8;
   constexpr int GPB = kPoolThreads / G;
   constexpr int W = ipow(P, L - 1);
-  constexpr int TB = (W < 8) ? W : 8;  // tokens loaded per batch (a multiple of P)
+  constexpr int TB = pool_batch(W);  // tokens per batch (a multiple of P)
+  constexpr int NB = W / TB;          // batches per block
   static_assert(TB % P == 0, "batch must hold whole level-1 entries");
+  extern __shared__ uint4 s_raw[];    // [kPoolStages][TB][kPoolThreads]
 
   const PoolJob& job = jobs.job[blockIdx.y];
   const int lane = threadIdx.x % G;
@@ -72,44 +112,113 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
 
   const __nv_bfloat16* xrow =
       reinterpret_cast<const __nv_bfloat16*>(job.x) + ((int64_t)bh * dm.N + (int64_t)blk * W) * D + lane * 8;
-  float* scores = job.scores ? job.scores + (int64_t)bh * dm.Rs : nullptr;
+  float* scores = kScore ? job.scores + (int64_t)bh * dm.Rs : nullptr;  // jobs with scores run as kScore
   __nv_bfloat16* pyr = reinterpret_cast<__nv_bfloat16*>(job.pyr);
 
-  double acc[L][8];  // acc[l]: running sum of the current level-l entry (l >= 1)
+  double acc[L][8];  // acc[l]: running fp64 sum of the current level-l entry (l >= 1)
 
-#pragma unroll 1
-  for (int t0 = 0; t0 < W; t0 += TB) {
-    uint4 raw[TB];
+  uint4* my = s_raw + threadIdx.x;  // this thread's slot u of stage st: my[(st * TB + u) * kPoolThreads]
+  auto issue = [&](int bi) {
+    const int st = bi % kPoolStages;
 #pragma unroll
-    for (int u = 0; u < TB; ++u) raw[u] = ld_stream16(xrow + (int64_t)(t0 + u) * D);
+    for (int u = 0; u < TB; ++u)
+      cp_async16(smem_u32(my + (st * TB + u) * kPoolThreads), xrow + (int64_t)(bi * TB + u) * D);
+  };
+#pragma unroll
+  for (int bi = 0; bi < kPoolStages - 1; ++bi) {
+    if (bi < NB) issue(bi);
+    cp_async_commit();
+  }
+#pragma unroll 1
+  for (int bi = 0; bi < NB; ++bi) {
+    if (bi + kPoolStages - 1 < NB) issue(bi + kPoolStages - 1);
+    cp_async_commit();
+    cp_async_wait<kPoolStages - 1>();  // batch bi has landed in this thread's slots
+    const int t0 = bi * TB;
+    const uint4* raw_s = my + (bi % kPoolStages) * TB * kPoolThreads;  // row u at raw_s[u * kPoolThreads]
 
 #pragma unroll
     for (int g1 = 0; g1 < TB / P; ++g1) {
+      float up[8], dn[8];
 #pragma unroll
       for (int c = 0; c < P; ++c) {
-        double x[8];
-        load_row8(raw[g1 * P + c], x);
-        if (scores) {  // level 0 is scored whenever L >= 2
+        float xf[8];
+        unpack8(raw_s[(g1 * P + c) * kPoolThreads], xf);
+        if (kScore) {  // level 0 is scored whenever L >= 2
+          double x[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = (double)xf[i];
           float s = row_score<G>(x);
           if (active && lane == 0) scores[dm.off[0] + (int64_t)blk * W + t0 + g1 * P + c] = s;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[1][i] = (c == 0) ? x[i] : acc[1][i] + x[i];
+        for (int i = 0; i < 8; ++i) {
+          up[i] = (c == 0) ? xf[i] : add_up(up[i], xf[i]);
+          dn[i] = (c == 0) ? xf[i] : add_dn(dn[i], xf[i]);
+        }
       }
-      // level-1 entry complete; walk up while parents complete
+      bool exact = true;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) exact &= same_sum(up[i], dn[i]);
+      const int j1 = blk * (W / P) + t0 / P + g1;  // global level-1 index
+      const bool write1 = (job.write_mask >> 1) & 1u;
+      const bool score1 = kScore && 1 <= L - 2;
+      // the fp64 level-1 sum: needed above level 1, and for the rounding when the fp32 one is not exact
+      if (!exact) {
+#pragma unroll
+        for (int c = 0; c < P; ++c) {
+          double x[8];
+          load_row8(raw_s[(g1 * P + c) * kPoolThreads], x);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[1][i] = (c == 0) ? x[i] : acc[1][i] + x[i];
+        }
+      } else if (L > 2) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[1][i] = (double)up[i];
+      }
+      if (write1 || score1) {
+        uint4 packed;
+        bool fast = exact;
+        float pv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pv[i] = mul_rn(up[i], 1.0f / (float)P);  // exact scaling by a power of two while the result is normal
+          fast &= zero_or_normal(pv[i]);
+        }
+        if (fast) {
+          packed = make_uint4(pack_bf16x2_rn(pv[0], pv[1]), pack_bf16x2_rn(pv[2], pv[3]),
+                              pack_bf16x2_rn(pv[4], pv[5]), pack_bf16x2_rn(pv[6], pv[7]));
+        } else {
+          if (exact && L <= 2) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[1][i] = (double)up[i];
+          }
+          double unused[8];
+          packed = round_pooled(acc[1], 1.0 / (double)P, unused);
+        }
+        if (write1 && active) st16(pyr + ((int64_t)bh * job.pyr_rows + job.row_off[1] + j1) * D + lane * 8, packed);
+        if (score1) {
+          float vf[8];
+          unpack8(packed, vf);
+          double v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = (double)vf[i];
+          const float sc = row_score<G>(v);
+          if (active && lane == 0) scores[dm.off[1] + j1] = sc;
+        }
+      }
+      // levels >= 2: walk up while parents complete
       int jloc = t0 / P + g1;  // index of the completed level-1 entry inside this block
 #pragma unroll
-      for (int lev = 1; lev < L; ++lev) {
-        if (lev > 1) {
-          const int c = jloc % P;  // child index of the completed level-(lev-1) entry
+      for (int lev = 2; lev < L; ++lev) {
+        const int c = jloc % P;  // child index of the completed level-(lev-1) entry
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[lev][i] = (c == 0) ? acc[lev - 1][i] : acc[lev][i] + acc[lev - 1][i];
-          if (c != P - 1) break;
-          jloc /= P;
-        }
+        for (int i = 0; i < 8; ++i) acc[lev][i] = (c == 0) ? acc[lev - 1][i] : acc[lev][i] + acc[lev - 1][i];
+        if (c != P - 1) break;
+        jloc /= P;
         const int64_t j = (int64_t)blk * (W / ipow(P, lev)) + jloc;  // global index at level lev
         const bool write = (job.write_mask >> lev) & 1u;
-        const bool score = scores && lev <= L - 2;
+        const bool score = kScore && lev <= L - 2;
         if (write || score) {
           double val[8];
           const uint4 packed = round_pooled(acc[lev], 1.0 / (double)ipow(P, lev), val);
@@ -198,15 +307,32 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherJobs jobs, const int3
   st16(reinterpret_cast<__half*>(job.out) + row * D + lane * 8, h);
 }
 
-template <int D, int P, int L>
-int launch_pool_t(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+// Jobs with scores and jobs without run as two launches of the two specialisations (the one without carries no
+// scoring code and fewer registers).
+template <int D, int P, int L, bool kScore>
+int launch_pool_kind(const PoolJobs& all, int njobs, const LhDims& dm, cudaStream_t st) {
+  PoolJobs jobs;
+  int n = 0;
+  for (int i = 0; i < njobs; ++i)
+    if ((all.job[i].scores != nullptr) == kScore) jobs.job[n++] = all.job[i];
+  if (n == 0) return LH_OK;
   constexpr int G = D / 8;
   constexpr int W = ipow(P, L - 1);
   const int64_t groups = (int64_t)dm.BH * (dm.N / W);
   const int64_t blocks = (groups + kPoolThreads / G - 1) / (kPoolThreads / G);
   if (blocks > 0x7fffffff) return LH_ERR_UNSUPPORTED;
-  pool_score_kernel<D, P, L><<<dim3((unsigned)blocks, njobs), kPoolThreads, 0, st>>>(jobs, dm);
+  const int smem = kPoolStages * pool_batch(W) * kPoolThreads * (int)sizeof(uint4);
+  auto kernel = pool_score_kernel<D, P, L, kScore>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return LH_ERR_CUDA;
+  kernel<<<dim3((unsigned)blocks, n), kPoolThreads, smem, st>>>(jobs, dm);
   return check_launch();
+}
+
+template <int D, int P, int L>
+int launch_pool_t(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
+  const int rc = launch_pool_kind<D, P, L, false>(jobs, njobs, dm, st);
+  return rc != LH_OK ? rc : launch_pool_kind<D, P, L, true>(jobs, njobs, dm, st);
 }
 
 template <int D, int P>
