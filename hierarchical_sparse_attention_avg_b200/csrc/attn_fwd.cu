@@ -187,31 +187,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(Lay::B_SE + b));  // score buffer b may be overwritten by S_{j+2}
 
-      const bool diag = (j == qt);
-      float mx = -INFINITY;
+      // row max of the raw scores (the scale is positive), as 8 independent chains; keys above the diagonal of
+      // the last tile are masked first
+      if (j == qt) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > row) s[c][i] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(s[0][k], s[0][k + 8]);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float x = s[c][i] * scale_log2;
-          if (diag && (c * 32 + i) > row) x = -INFINITY;
-          s[c][i] = x;
-          mx = fmaxf(mx, x);
-        }
+        for (int i = 0; i < 32; ++i)
+          if (c > 0 || i >= 16) mx8[i & 7] = fmaxf(mx8[i & 7], s[c][i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
       const float m_new = fmaxf(m_run, mx);
       l_run *= ex2(m_run - m_new);  // 1 without growth; 0 on the first tile
       m_run = m_new;
-      // P of this tile (fp16, in [0, 1]) and its row sum
+      // P of this tile (fp16, in [0, 1]) = 2^(s * scale - m) and its row sum (8 independent chains)
       uint32_t pk[64];
-      float rs = 0.f;
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2(s[c][i] - m_run), p1 = ex2(s[c][i + 1] - m_run);
-          rs += p0 + p1;
+          const float p0 = ex2(fmaf(s[c][i], scale_log2, -m_run)), p1 = ex2(fmaf(s[c][i + 1], scale_log2, -m_run));
+          rs8[(i >> 1) & 7] += p0 + p1;
           pk[c * 16 + i / 2] = pack_half2_rn(p0, p1);
         }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l_run += rs;
       // O_b and P buffer b are free once the product of tile j-2 has completed
       if (j >= 2) {
