@@ -200,14 +200,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* s_lse = reinterpret_cast<float*>(smem + Lay::STAT);
     float* s_d = s_lse + 2 * kQTile;
     bool ok = true;
+    // statistics (LSE and D) of one query each, loaded one sub-tile ahead so that their latency is hidden
+    auto load_stats = [&](int i, float& l, float& dd) {
+      const int q = i * kQTile + ct;
+      l = (ct < kQTile && q < S) ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
+      dd = (ct < kQTile && q < S) ? dvec[(int64_t)bh * S + q] : 0.f;
+    };
+    float nl = INFINITY, nd = 0.f;
+    if (nit > 0) load_stats(i0, nl, nd);
     for (int it = 0; it < nit; ++it) {
       const int b = it & 1, i = i0 + it;
       // statistics of the sub-tile into buffer b (its previous readers, sub-tile it-2, are done: same threads)
       if (ct < kQTile) {
-        const int q = i * kQTile + ct;
-        s_lse[b * kQTile + ct] = q < S ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
-        s_d[b * kQTile + ct] = q < S ? dvec[(int64_t)bh * S + q] : 0.f;
+        s_lse[b * kQTile + ct] = nl;
+        s_d[b * kQTile + ct] = nd;
       }
+      if (it + 1 < nit) load_stats(i + 1, nl, nd);
       ok = named_barrier_and(kBarCompute, 128, ok);
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_abort, status));
@@ -221,23 +229,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
       }
       uint32_t pk[32], dk[32];
-      float ds_max = 0.f;
       if (ok) {
+        float dsm[4] = {0.f, 0.f, 0.f, 0.f};  // largest |dS| as 4 independent chains
+        const bool diag = i * kQTile < key;  // some query of the sub-tile precedes the key (masked)
 #pragma unroll
         for (int c = 0; c < kQTile; c += 2) {
           float p2[2], d2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int q = i * kQTile + c + e;
-            float pv = ex2(sv[c + e] * scale_log2 - s_lse[b * kQTile + c + e]);
-            if (q < key) pv = 0.f;  // query q does not see key `key`
+            float pv = ex2(fmaf(sv[c + e], scale_log2, -s_lse[b * kQTile + c + e]));
+            if (diag && i * kQTile + c + e < key) pv = 0.f;  // query does not see key `key`
             p2[e] = pv;
             d2[e] = pv * (dp[c + e] - s_d[b * kQTile + c + e]) * scale;
-            ds_max = fmaxf(ds_max, fabsf(d2[e]));
+            dsm[(c / 2) & 3] = fmaxf(dsm[(c / 2) & 3], fabsf(d2[e]));
           }
           pk[c / 2] = pack_half2_rn(p2[0], p2[1]);
           dk[c / 2] = pack_half2_rn(d2[0], d2[1]);
         }
+        const float ds_max = fmaxf(fmaxf(dsm[0], dsm[1]), fmaxf(dsm[2], dsm[3]));
         if (__any_sync(0xffffffffu, !(ds_max <= 65504.f)) && lane == 0) set_status(status, LH_ERR_RANGE);
         // P/dS buffer b is free once the products of sub-tile it-2 have completed
         if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_abort,
