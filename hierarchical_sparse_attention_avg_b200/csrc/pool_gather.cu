@@ -234,20 +234,76 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
   }
 }
 
-template <int D, int P, int LEV>
-__device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8]) {
-  if constexpr (LEV == 0) {
-    load_row8(ld16(p), out);
-  } else if constexpr (ipow(P, LEV) <= 16) {
-    // few enough rows to keep all of their loads in flight at once; the sums keep the tree order
-    constexpr int CW = ipow(P, LEV - 1);
+// Level-1 entry of P raw rows (already loaded) summed with the exact fp32 chains described above; the result
+// tells whether the chains agree (then `up` is the sum the definition fixes).
+template <int P>
+__device__ __forceinline__ bool level1_f32(const uint4* raw, float (&up)[8]) {
+  float dn[8];
+#pragma unroll
+  for (int c = 0; c < P; ++c) {
+    float x[8];
+    unpack8(raw[c], x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      up[i] = (c == 0) ? x[i] : add_up(up[i], x[i]);
+      dn[i] = (c == 0) ? x[i] : add_dn(dn[i], x[i]);
+    }
+  }
+  bool exact = true;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) exact &= same_sum(up[i], dn[i]);
+  return exact;
+}
+
+// fp64 sum of the level-LEV entry at p in the definition's tree order: level-1 sums from the fp32 chains when
+// exact (one widening per entry), else in fp64 from the raw values.
+template <int P>
+__device__ __forceinline__ void level1_f64(const uint4* raw, double (&out)[8]) {
+  float up[8];
+  if (level1_f32<P>(raw, up)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = (double)up[i];
+  } else {
+#pragma unroll
+    for (int c = 0; c < P; ++c) {
+      double x[8];
+      load_row8(raw[c], x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? x[i] : out[i] + x[i];
+    }
+  }
+}
+
+// The tree over raw rows already in registers (P^LEV of them).
+template <int P, int LEV>
+__device__ __forceinline__ void tree_from_raw(const uint4* raw, double (&out)[8]) {
+  if constexpr (LEV == 1) {
+    level1_f64<P>(raw, out);
+  } else {
 #pragma unroll
     for (int c = 0; c < P; ++c) {
       double ch[8];
-      tree_sum<D, P, LEV - 1>(p + (int64_t)c * CW * D, ch);
+      tree_from_raw<P, LEV - 1>(raw + c * ipow(P, LEV - 1), ch);
 #pragma unroll
       for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? ch[i] : out[i] + ch[i];
     }
+  }
+}
+
+template <int D, int P, int LEV>
+__device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8]) {
+  if constexpr (ipow(P, LEV) <= 16) {
+    // few enough rows to keep all of their loads in flight at once; the sums keep the tree order
+    constexpr int R = ipow(P, LEV);
+    uint4 raw[R];
+#pragma unroll
+    for (int u = 0; u < R; ++u) raw[u] = ld16(p + (int64_t)u * D);
+    tree_from_raw<P, LEV>(raw, out);
+  } else if constexpr (LEV == 1) {
+    uint4 raw[P];
+#pragma unroll
+    for (int u = 0; u < P; ++u) raw[u] = ld16(p + (int64_t)u * D);
+    level1_f64<P>(raw, out);
   } else {
     constexpr int CW = ipow(P, LEV - 1);
 #pragma unroll 1
@@ -260,15 +316,32 @@ __device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8
   }
 }
 
-// Pooled value of entry (lev, j) recomputed from the raw rows with the same summation tree as the pool kernel.
+// Pooled (bf16) value of entry (lev, j) recomputed from the raw rows with the same summation tree as the pool
+// kernel: a level-1 entry whose fp32 chains agree is rounded straight from fp32.
 template <int D, int P>
 __device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
   double s[8], val[8];
-  switch (lev) {
-    case 1: tree_sum<D, P, 1>(x0, s); break;
-    case 2: tree_sum<D, P, 2>(x0, s); break;
-    case 3: tree_sum<D, P, 3>(x0, s); break;
-    default: tree_sum<D, P, 4>(x0, s); break;
+  if (lev == 1) {
+    uint4 raw[P];
+#pragma unroll
+    for (int u = 0; u < P; ++u) raw[u] = ld16(x0 + (int64_t)u * D);
+    float up[8], pv[8];
+    bool fast = level1_f32<P>(raw, up);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      pv[i] = mul_rn(up[i], 1.0f / (float)P);
+      fast &= zero_or_normal(pv[i]);
+    }
+    if (fast)
+      return make_uint4(pack_bf16x2_rn(pv[0], pv[1]), pack_bf16x2_rn(pv[2], pv[3]), pack_bf16x2_rn(pv[4], pv[5]),
+                        pack_bf16x2_rn(pv[6], pv[7]));
+    tree_sum<D, P, 1>(x0, s);
+  } else if (lev == 2) {
+    tree_sum<D, P, 2>(x0, s);
+  } else if (lev == 3) {
+    tree_sum<D, P, 3>(x0, s);
+  } else {
+    tree_sum<D, P, 4>(x0, s);
   }
   return round_pooled(s, 1.0 / (double)ipow(P, lev), val);
 }
@@ -277,7 +350,7 @@ __device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
 // it as fp16, the operand format of the attention kernels (every bf16 value of magnitude in [2^-14, 65504] is
 // exact in fp16; a larger one records LH_ERR_RANGE).
 template <int D, int P>
-__global__ void __launch_bounds__(256) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
+__global__ void __launch_bounds__(256, 2) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
                                                      LhDims dm) {
   constexpr int G = D / 8;
   const GatherJob& job = jobs.job[blockIdx.y];
