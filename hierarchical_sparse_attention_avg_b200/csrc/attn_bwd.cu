@@ -11,7 +11,9 @@
 //   warp 1     MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into one of two TMEM buffer pairs,
 //              then, for the previous sub-tile, dV += P^T dO, dK += dS^T Q (accumulated in TMEM for the whole
 //              loop) and dQ^T = K_j^T dS^T (into the consumed S^T columns);
-//   warps 2-5  compute: one key row (TMEM lane) per thread writes the P^T and dS^T rows (fp16) of the sub-tile;
+//   warps 2-5  compute: one key row (TMEM lane) per thread writes the P^T and dS^T rows (fp16) of the sub-tile
+//              to tensor memory, over the S^T and dP^T columns they came from (there they are the A operands of
+//              dV += P^T dO and dK += dS^T Q), and dS^T also to shared memory (the B operand of dQ^T);
 //   warps 6-9  drain: one feature (TMEM lane) per thread moves dQ^T out of TMEM into a shared-memory tile that
 //              one thread adds to the fp32 dQ accumulator with TMA bulk tensor reduce-add.
 // The MMA thread issues S^T/dP^T of sub-tile i+1 before the products of sub-tile i, so the tensor core works while
@@ -44,8 +46,7 @@ struct BwdLayout {
   static constexpr uint32_t V = KT;
   static constexpr uint32_t Q = 2 * KT;                      // kStages
   static constexpr uint32_t DO = Q + kStages * QT;           // kStages
-  static constexpr uint32_t P = DO + kStages * QT;           // 2 buffers
-  static constexpr uint32_t DS = P + 2 * PT;                 // 2 buffers
+  static constexpr uint32_t DS = DO + kStages * QT;          // 2 buffers (dS^T, the B operand of dQ^T)
   static constexpr uint32_t DQ = DS + 2 * PT;                // staging: [d/32][64 q][32 f] fp32
   static constexpr uint32_t STAT = DQ + kQTile * D * 4;      // [2][64] LSE*log2e, [2][64] D
   static constexpr uint32_t BAR = STAT + 4 * kQTile * 4;
@@ -148,15 +149,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = jt & 1, s = jt % kStages;
         if (!mbar_wait(bar(Lay::B_DSF + b), (jt >> 1) & 1, &s_abort, status)) return false;
         tc_fence_after();
-        const uint32_t sP = sb + Lay::P + b * Lay::PT, sDS = sb + Lay::DS + b * Lay::PT;
+        const uint32_t sDS = sb + Lay::DS + b * Lay::PT;
         const uint32_t sQ = sb + Lay::Q + s * Lay::QT, sDO = sb + Lay::DO + s * Lay::QT;
+        // P^T and dS^T (fp16 pairs) sit over the first 32 columns of the S^T and dP^T buffers
+        const uint32_t tP = tmem + 128 * b, tDS = tmem + 128 * b + 64;
 #pragma unroll
         for (int kk = 0; kk < kQTile / 16; ++kk) {  // reduction over the 64 queries
           const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
-          umma_ss(tDV, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sDO + kk * 2048, 8192, 1024), idesc_acc,
-                  acc);
-          umma_ss(tDK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc,
-                  acc);
+          umma_ts(tDV, tP + kk * 8, sdesc_sw128(sDO + kk * 2048, 8192, 1024), idesc_acc, acc);
+          umma_ts(tDK, tDS + kk * 8, sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc, acc);
         }
 #pragma unroll
         for (int kk = 0; kk < kKTile / 16; ++kk)  // reduction over the 128 keys
@@ -253,15 +254,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                             status));
       }
       if (ok) {
-        uint8_t* sP = smem + Lay::P + b * Lay::PT;
+        // P^T and dS^T rows to tensor memory (A operands of dV and dK), dS^T also to shared memory (B of dQ^T)
+        float pf[32], df[32];
+#pragma unroll
+        for (int w = 0; w < 32; ++w) {
+          pf[w] = __uint_as_float(pk[w]);
+          df[w] = __uint_as_float(dk[w]);
+        }
+        tmem_st32(tmem + 128 * b + lane_base, pf);
+        tmem_st32(tmem + 128 * b + 64 + lane_base, df);
         uint8_t* sDS = smem + Lay::DS + b * Lay::PT;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunk ch holds queries 8 ch .. 8 ch + 7
           const uint32_t off = sw128_offset(r, ch);
-          *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
           *reinterpret_cast<uint4*>(sDS + off) = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
         }
         fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_DSF + b));
       }
