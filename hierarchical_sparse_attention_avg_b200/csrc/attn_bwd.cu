@@ -33,7 +33,7 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kKTile = 128;  // key rows per CTA
 constexpr int kQTile = 64;   // query rows per sub-tile
-constexpr int kStages = 2;   // Q/dO ring depth
+constexpr int kStages = 3;   // Q/dO ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBarCompute = 1, kBarDrain = 2;  // named barrier ids (0 is __syncthreads)
 
