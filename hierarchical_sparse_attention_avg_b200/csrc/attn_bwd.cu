@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto load_stats = [&](int i, float& l, float& dd) {
       const int q = i * kQTile + ct;
       l = (ct < kQTile && q < S) ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
-      dd = (ct < kQTile && q < S) ? dvec[(int64_t)bh * S + q] : 0.f;
+      dd = (ct < kQTile && q < S) ? dvec[(int64_t)bh * S + q] * scale : 0.f;  // D already times the scale
     };
     float nl = INFINITY, nd = 0.f;
     if (nit > 0) load_stats(i0, nl, nd);
@@ -231,8 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t pk[32], dk[32];
       if (ok) {
-        float dsm[4] = {0.f, 0.f, 0.f, 0.f};  // largest |dS| as 4 independent chains
         const bool diag = i * kQTile < key;  // some query of the sub-tile precedes the key (masked)
+        // dS = P (dP - D) scale = P fma(dP, scale, -D scale); the fp16 range is checked on the packed values (a
+        // value beyond it became an infinity, NaN stays NaN): largest |dS| half2 over 4 independent chains
+        __half2 hm[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) hm[k] = __float2half2_rn(0.f);
 #pragma unroll
         for (int c = 0; c < kQTile; c += 2) {
           float p2[2], d2[2];
@@ -241,14 +245,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             float pv = ex2(fmaf(sv[c + e], scale_log2, -s_lse[b * kQTile + c + e]));
             if (diag && i * kQTile + c + e < key) pv = 0.f;  // query does not see key `key`
             p2[e] = pv;
-            d2[e] = pv * (dp[c + e] - s_d[b * kQTile + c + e]) * scale;
-            dsm[(c / 2) & 3] = fmaxf(dsm[(c / 2) & 3], fabsf(d2[e]));
+            d2[e] = pv * fmaf(dp[c + e], scale, -s_d[b * kQTile + c + e]);
           }
           pk[c / 2] = pack_half2_rn(p2[0], p2[1]);
           dk[c / 2] = pack_half2_rn(d2[0], d2[1]);
+          const __half2 h = *reinterpret_cast<const __half2*>(&dk[c / 2]);
+          hm[(c / 2) & 3] = __hmax2_nan(hm[(c / 2) & 3], __habs2(h));
         }
-        const float ds_max = fmaxf(fmaxf(dsm[0], dsm[1]), fmaxf(dsm[2], dsm[3]));
-        if (__any_sync(0xffffffffu, !(ds_max <= 65504.f)) && lane == 0) set_status(status, LH_ERR_RANGE);
+        const __half2 h01 = __hmax2_nan(hm[0], hm[1]), h23 = __hmax2_nan(hm[2], hm[3]);
+        const float2 mf = __half22float2(__hmax2_nan(h01, h23));
+        if (__any_sync(0xffffffffu, !(mf.x <= 65504.f && mf.y <= 65504.f)) && lane == 0)
+          set_status(status, LH_ERR_RANGE);
         // P/dS buffer b is free once the products of sub-tile it-2 have completed
         if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_abort,
                                                             status));
