@@ -237,15 +237,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         __half2 hm[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) hm[k] = __float2half2_rn(0.f);
+        // the sub-tile's statistics as 16-byte vectors (the same for every thread: broadcast loads)
+        const float4* sl4 = reinterpret_cast<const float4*>(s_lse + b * kQTile);
+        const float4* sd4 = reinterpret_cast<const float4*>(s_d + b * kQTile);
 #pragma unroll
         for (int c = 0; c < kQTile; c += 2) {
           float p2[2], d2[2];
+          const float4 l4 = sl4[c >> 2], d4 = sd4[c >> 2];
+          const float lv[2] = {(c & 2) ? l4.z : l4.x, (c & 2) ? l4.w : l4.y};
+          const float dv[2] = {(c & 2) ? d4.z : d4.x, (c & 2) ? d4.w : d4.y};
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            float pv = ex2(fmaf(sv[c + e], scale_log2, -s_lse[b * kQTile + c + e]));
+            float pv = ex2(fmaf(sv[c + e], scale_log2, -lv[e]));
             if (diag && i * kQTile + c + e < key) pv = 0.f;  // query does not see key `key`
             p2[e] = pv;
-            d2[e] = pv * fmaf(dp[c + e], scale, -s_d[b * kQTile + c + e]);
+            d2[e] = pv * fmaf(dp[c + e], scale, -dv[e]);
           }
           pk[c / 2] = pack_half2_rn(p2[0], p2[1]);
           dk[c / 2] = pack_half2_rn(d2[0], d2[1]);
