@@ -73,6 +73,39 @@ def kernel_work(w: dict) -> dict:
     }, S
 
 
+# DRAM traffic per launch from a one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), recorded in
+# profiles/dram_traffic.txt with a digest of the kernel's sources; reported only while the sources still match.
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic.txt")
+CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "hierarchical_sparse_attention_avg_b200", "csrc")
+KERNEL_SOURCES = {"attn_bwd": "attn_bwd.cu", "attn_fwd": "attn_fwd.cu", "pool_score": "pool_gather.cu",
+                  "gather": "pool_gather.cu", "unpool_bwd": "scatter.cu", "scatter": "scatter.cu",
+                  "scatter_bwd": "scatter.cu", "bwd_prep": "scatter.cu", "absmax": "scatter.cu", "topk": "topk.cu",
+                  "order": "topk.cu"}
+
+
+def source_digest(kernel: str) -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in (KERNEL_SOURCES.get(kernel, ""), "lh_common.cuh", "internal.h", "api.cu"):
+        path = os.path.join(CSRC, f)
+        if f and os.path.exists(path):
+            h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """Bytes per launch (read + write) of `kernel` at `workload`, or None when not captured for these sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    for line in open(TRAFFIC_FILE):
+        f = line.split()
+        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
+            if f[4] == source_digest(kernel):
+                return int(f[2]) + int(f[3])
+    return None
+
+
 class NvmlClockSampler:
     """SM clock and clock-event reasons read through NVML every 10 ms in a thread while the timed region runs
     (read-only queries; no setting of the GPU is changed)."""
@@ -363,7 +396,7 @@ def main():
     tname, tk = top
     roofline = {"kernel": tname, "bound": tk["bound"], "achieved": tk["achieved"],
                 "peak": peaks["bf16_sust"] if tk["bound"] == "tensor" else peaks["hbm"], "unit": tk["unit"],
-                "frac": tk["frac"], "traffic": None,
+                "frac": tk["frac"], "traffic": measured_traffic(tname, args.workload),
                 "peak_source": f"{peaks['src']} ({'bf16 sustained' if tk['bound'] == 'tensor' else 'HBM copy'})"}
     gpu_launches = sum(v_[0] for v_ in prof.values())
 
