@@ -349,13 +349,17 @@ __device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
 // One group per gathered row (b, h, s): copy (level 0), read (pyramid) or recompute (pooled) the row, and store
 // it as fp16, the operand format of the attention kernels (every bf16 value of magnitude in [2^-14, 65504] is
 // exact in fp16; a larger one records LH_ERR_RANGE).
+// Small blocks (kGatherThreads), many per SM: rows cost from one to p^(L-2) raw rows, and a block retires only
+// with its slowest row.
+constexpr int kGatherThreads = 32;
+
 template <int D, int P>
-__global__ void __launch_bounds__(256, 2) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
-                                                     LhDims dm) {
+__global__ void __launch_bounds__(kGatherThreads, 16) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
+                                                                 LhDims dm) {
   constexpr int G = D / 8;
   const GatherJob& job = jobs.job[blockIdx.y];
   const int lane = threadIdx.x % G;
-  const int64_t row = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
+  const int64_t row = (int64_t)blockIdx.x * (kGatherThreads / G) + threadIdx.x / G;
   if (row >= (int64_t)dm.BH * dm.S) return;
   const int bh = (int)(row / dm.S);
   const int gid = idx_g[row];
@@ -435,12 +439,12 @@ template <int D>
 int launch_gather_d(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st) {
   constexpr int G = D / 8;
   const int64_t rows = (int64_t)dm.BH * dm.S;
-  const int64_t blocks = (rows + 256 / G - 1) / (256 / G);
+  const int64_t blocks = (rows + kGatherThreads / G - 1) / (kGatherThreads / G);
   dim3 grid((unsigned)blocks, njobs);
   switch (dm.p) {
-    case 2: gather_kernel<D, 2><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
-    case 4: gather_kernel<D, 4><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
-    case 8: gather_kernel<D, 8><<<grid, 256, 0, st>>>(jobs, idx_g, dm); break;
+    case 2: gather_kernel<D, 2><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
+    case 4: gather_kernel<D, 4><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
+    case 8: gather_kernel<D, 8><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
     default: return LH_ERR_UNSUPPORTED;
   }
   return check_launch();
