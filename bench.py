@@ -31,6 +31,11 @@ WORKLOADS = {
     "stress1M": dict(B=1, H=8, N=1048576, d=128, L=4, p=4, k=4096, C=32),
     # a smaller d=128 case with the long-context level structure, for profiler captures that must stay small
     "probe128K": dict(B=1, H=4, N=131072, d=128, L=4, p=4, k=4096, C=32),
+    # dense comparator: one level, identity selection (S = N), i.e. plain causal attention through the same kernels
+    "dense512K": dict(B=1, H=16, N=524288, d=128, L=1, p=4, k=1, C=1),
+    # variant parameters: the recipe's L=3, k=1536, and the ablation grid's L in {3, 4}, k in {1536, 2048} at 98K
+    "recipe98K": dict(B=1, H=16, N=98304, d=64, L=3, p=4, k=1536, C=16),
+    "ablation98K_L4k1536": dict(B=1, H=16, N=98304, d=64, L=4, p=4, k=1536, C=16),
 }
 DEFAULT_WORKLOAD = "long512K"
 METRIC = "Lighthouse fwd+bwd tokens/s at N=512K; HBM GB/s and attention TFLOP/s vs peak"
