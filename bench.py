@@ -224,6 +224,21 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise max of `values` (floats) over all ranks.  Every rank calls it at the same points, in the same
+    order, including on error paths (a device status is reduced with the times, so all ranks raise together)."""
+    if world == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tokens(w: dict, world: int) -> int:
+    """Tokens all ranks process in one step: each rank runs its own batch (weak scaling)."""
+    return w["B"] * w["N"] * world
+
+
 def cpu_baseline(w: dict, seed: int = 0) -> dict:
     """The CPU oracle timed on one head of the workload (forward + backward), scaled to tokens/s of the whole
     workload (heads are independent, so the time of all B*H heads is B*H times one head's)."""
@@ -332,18 +347,15 @@ def main():
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
     lh.lh_profile_enable(False)
     prof = lh.lh_profile_read()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    status = lh.lh_get_status(dev)
+    ms, status = max_over_ranks([e0.elapsed_time(e1) / args.steps, lh.lh_get_status(dev)], world, dev)
     if status != 0:
-        raise RuntimeError(f"device status {status}: {lh.error_string(status)}")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    tokens = w["B"] * w["N"] * world
+        raise RuntimeError(f"device status {int(status)}: {lh.error_string(int(status))}")
+    tokens = whole_job_tokens(w, world)
     value = tokens / (ms / 1e3)
 
     # end to end through the C ABI with host buffers: H2D of the step's inputs, the step, D2H of its outputs
@@ -372,11 +384,9 @@ def main():
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = a0.elapsed_time(a1) / n_e2e
         if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+            torch.distributed.barrier()
+        ms_e2e = max_over_ranks([a0.elapsed_time(a1) / n_e2e], world, dev)[0]
         nbytes = sum(t.numel() * t.element_size() for t in host_in)
         obytes = sum(t.numel() * t.element_size() for t in host_out)
         e2e = {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
