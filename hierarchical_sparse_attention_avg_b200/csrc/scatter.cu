@@ -343,14 +343,19 @@ __global__ void __launch_bounds__(kWinThreads, 4) window_sum_kernel(const float*
   cp_async_wait<0>();
 }
 
+// Small blocks (many per SM) for the scatter backward: a gathered row sums a window of 1 to p^(L-1) upstream rows,
+// and a block retires only with its slowest row.
+constexpr int kSbThreads = 64;
+
 template <int D>
-__global__ void __launch_bounds__(256) scatter_bwd_kernel(const __nv_bfloat16* __restrict__ dout,
-                                                          const int32_t* __restrict__ idx_g, float* __restrict__ dog,
-                                                          unsigned int* __restrict__ amax, LhDims dm) {
+__global__ void __launch_bounds__(kSbThreads) scatter_bwd_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                                 const int32_t* __restrict__ idx_g,
+                                                                 float* __restrict__ dog,
+                                                                 unsigned int* __restrict__ amax, LhDims dm) {
   constexpr int G = D / 8;
   const int lane = threadIdx.x % G;
   const int64_t total = (int64_t)dm.BH * dm.S;
-  const int64_t row0 = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
+  const int64_t row0 = (int64_t)blockIdx.x * (kSbThreads / G) + threadIdx.x / G;
   const bool active = row0 < total;
   const int64_t row = active ? row0 : total - 1;
   const int bh = (int)(row / dm.S);
@@ -363,12 +368,12 @@ __global__ void __launch_bounds__(256) scatter_bwd_kernel(const __nv_bfloat16* _
   const __nv_bfloat16* src = dout + ((int64_t)bh * dm.N) * D + lane * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int t = t0;
-  for (; t + 3 <= t1; t += 4) {  // four rows in flight
-    uint4 r[4];
+  for (; t + 7 <= t1; t += 8) {  // eight rows in flight
+    uint4 r[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) r[u] = ld_stream16(src + (int64_t)(t + u) * D);
+    for (int u = 0; u < 8; ++u) r[u] = ld_stream16(src + (int64_t)(t + u) * D);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       float f[8];
       unpack8(r[u], f);
 #pragma unroll
@@ -498,9 +503,11 @@ int launch_scatter_bwd(const void* dout, const int32_t* idx_g, float* dog, unsig
   const int64_t rows = (int64_t)dm.BH * dm.S;
   KernelTimer timer("scatter_bwd", st);
   if (dm.d == 64)
-    scatter_bwd_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
+    scatter_bwd_kernel<64><<<(unsigned)((rows + kSbThreads / 8 - 1) / (kSbThreads / 8)), kSbThreads, 0, st>>>(
+        (const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
   else
-    scatter_bwd_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>((const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
+    scatter_bwd_kernel<128><<<(unsigned)((rows + kSbThreads / 16 - 1) / (kSbThreads / 16)), kSbThreads, 0, st>>>(
+        (const __nv_bfloat16*)dout, idx_g, dog, amax, dm);
   return check_launch();
 }
 
