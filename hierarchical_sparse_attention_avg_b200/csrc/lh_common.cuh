@@ -94,15 +94,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// fp32 <-> fp64 conversions that keep subnormal values whatever the compiler's flush-to-zero setting (the library
+// is built with fast math, which would otherwise flush them in C++ conversions).
+__device__ __forceinline__ double f64_of(float x) {
+  double r;
+  asm("cvt.f64.f32 %0, %1;" : "=d"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float f32_rn_of(double x) {
+  float r;
+  asm("cvt.rn.f32.f64 %0, %1;" : "=f"(r) : "d"(x));
+  return r;
+}
+__device__ __forceinline__ float f32_rz_of(double x) {
+  float r;
+  asm("cvt.rz.f32.f64 %0, %1;" : "=f"(r) : "d"(x));
+  return r;
+}
+
 // fp64 -> bf16 with a single round-to-nearest-even.  Method: round to fp32 toward zero, then make the result
 // "round to odd" by forcing its last bit when the conversion was inexact, then round that fp32 value to bf16
 // to nearest-even.  fp32 carries more than two extra bits over bf16, so the two steps equal one direct
 // rounding (Boldo & Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms using rounding
-// to odd", IEEE Trans. Computers 2008).
+// to odd", IEEE Trans. Computers 2008).  The last step is done on the bits (the bf16 conversion instruction
+// is not relied on for fp32 subnormals).
 __device__ __forceinline__ uint32_t f64_to_bf16_bits_rne(double x) {
-  float f = __double2float_rz(x);
-  if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+  uint32_t b = __float_as_uint(f32_rz_of(x));
+  if (f64_of(__uint_as_float(b)) != x) b |= 1u;
+  if ((b & 0x7F800000u) == 0x7F800000u) return (b >> 16) | ((b & 0xFFFFu) ? 0x40u : 0u);  // inf stays, NaN quiet
+  return (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;  // round to nearest, ties to even, on the bits
 }
 
 // ------------------------------------------------------------------------------------------------------------

@@ -28,7 +28,7 @@ __device__ __forceinline__ void load_row8(const uint4& raw, double (&x)[8]) {
   float f[8];
   unpack8(raw, f);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = (double)f[i];
+  for (int i = 0; i < 8; ++i) x[i] = f64_of(f[i]);
 }
 
 // Score of one row: squared l2 norm of the (bf16) values x, summed in the fixed order, rounded to fp32.
@@ -39,7 +39,7 @@ __device__ __forceinline__ float row_score(const double (&x)[8]) {
   for (int i = 1; i < 8; ++i) s = fma(x[i], x[i], s);  // x*x is exact in fp64: fma == add of the square
 #pragma unroll
   for (int off = 1; off < G; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  return __double2float_rn(s);
+  return f32_rn_of(s);
 }
 
 // Round 8 fp64 sums / w to bf16 (single rounding), returning packed bits and the bf16 values as fp64.
@@ -48,7 +48,7 @@ __device__ __forceinline__ uint4 round_pooled(const double (&sum)[8], double inv
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     b[i] = f64_to_bf16_bits_rne(sum[i] * inv_w);  // inv_w = 1/p^l is exact for power-of-two p
-    val[i] = (double)__uint_as_float(b[i] << 16);
+    val[i] = f64_of(__uint_as_float(b[i] << 16));
   }
   return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
 }
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
         if (kScore) {  // level 0 is scored whenever L >= 2
           double x[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = (double)xf[i];
+          for (int i = 0; i < 8; ++i) x[i] = f64_of(xf[i]);
           float s = row_score<G>(x);
           if (active && lane == 0) scores[dm.off[0] + (int64_t)blk * W + t0 + g1 * P + c] = s;
         }
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
         }
       } else if (L > 2) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[1][i] = (double)up[i];
+        for (int i = 0; i < 8; ++i) acc[1][i] = f64_of(up[i]);
       }
       if (write1 || score1) {
         uint4 packed;
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
         } else {
           if (exact && L <= 2) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[1][i] = (double)up[i];
+            for (int i = 0; i < 8; ++i) acc[1][i] = f64_of(up[i]);
           }
           double unused[8];
           packed = round_pooled(acc[1], 1.0 / (double)P, unused);
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
           unpack8(packed, vf);
           double v[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = (double)vf[i];
+          for (int i = 0; i < 8; ++i) v[i] = f64_of(vf[i]);
           const float sc = row_score<G>(v);
           if (active && lane == 0) scores[dm.off[1] + j1] = sc;
         }
@@ -234,154 +234,274 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
   }
 }
 
-// Level-1 entry of P raw rows (already loaded) summed with the exact fp32 chains described above; the result
-// tells whether the chains agree (then `up` is the sum the definition fixes).
-template <int P>
-__device__ __forceinline__ bool level1_f32(const uint4* raw, float (&up)[8]) {
-  float dn[8];
+// ---- Gather (step 4).  One warp per gathered row: lane i holds features [2*NW*i, 2*NW*i + 2*NW) (NW 32-bit
+// words: d=128 -> 8 bytes, d=64 -> 4 bytes), so a row's level decides the warp's path as a whole.
+
+// One lane's share of one row: 2*NW bf16 values.
+template <int NW>
+struct RowW {
+  uint32_t w[NW];
+};
+
+template <int NW>
+__device__ __forceinline__ RowW<NW> ld_roww(const __nv_bfloat16* p) {
+  RowW<NW> r;
+  if constexpr (NW == 2) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    r.w[0] = v.x;
+    r.w[1] = v.y;
+  } else {
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r.w[0]) : "l"(p));
+  }
+  return r;
+}
+
+// Packed pair of fp32 values (low word first), the operand of the sm_100a f32x2 instructions.
+__device__ __forceinline__ uint64_t f32x2_of_bf16x2(uint32_t w) {
+  return ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+}
+__device__ __forceinline__ uint64_t add2_up(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rp.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2_dn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float sub_rn(float a, float b) {  // no flush of subnormal results
+  float r;
+  asm("sub.rn.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Interval sums.  The sum of a level-LEV entry is carried twice in fp32, every addition rounded up in one copy and
+// down in the other, in the definition's tree order (p children left to right at every level, each child being
+// the sum of its own children).  Rounding is monotone, so the upper copy never falls below the exact sum and the
+// lower never rises above it, and a copy that rounded once stays strictly apart from it.  Equal copies therefore
+// mean that every partial sum of the tree is exact in fp32 -- hence also in fp64, where the definition takes them
+// -- and that the common value is the sum the definition fixes.
+template <int NW, int P, int LEV>
+__device__ __forceinline__ void iv_regs(const RowW<NW>* raw, uint64_t (&up)[NW], uint64_t (&dn)[NW]) {
 #pragma unroll
   for (int c = 0; c < P; ++c) {
-    float x[8];
-    unpack8(raw[c], x);
+    uint64_t cu[NW], cd[NW];
+    if constexpr (LEV == 1) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      up[i] = (c == 0) ? x[i] : add_up(up[i], x[i]);
-      dn[i] = (c == 0) ? x[i] : add_dn(dn[i], x[i]);
+      for (int i = 0; i < NW; ++i) cu[i] = cd[i] = f32x2_of_bf16x2(raw[c].w[i]);
+    } else {
+      iv_regs<NW, P, LEV - 1>(raw + c * ipow(P, LEV - 1), cu, cd);
     }
-  }
-  bool exact = true;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) exact &= same_sum(up[i], dn[i]);
-  return exact;
-}
-
-// fp64 sum of the level-LEV entry at p in the definition's tree order: level-1 sums from the fp32 chains when
-// exact (one widening per entry), else in fp64 from the raw values.
-template <int P>
-__device__ __forceinline__ void level1_f64(const uint4* raw, double (&out)[8]) {
-  float up[8];
-  if (level1_f32<P>(raw, up)) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = (double)up[i];
-  } else {
-#pragma unroll
-    for (int c = 0; c < P; ++c) {
-      double x[8];
-      load_row8(raw[c], x);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? x[i] : out[i] + x[i];
+    for (int i = 0; i < NW; ++i) {
+      up[i] = c == 0 ? cu[i] : add2_up(up[i], cu[i]);
+      dn[i] = c == 0 ? cd[i] : add2_dn(dn[i], cd[i]);
     }
   }
 }
 
-// The tree over raw rows already in registers (P^LEV of them).
-template <int P, int LEV>
-__device__ __forceinline__ void tree_from_raw(const uint4* raw, double (&out)[8]) {
-  if constexpr (LEV == 1) {
-    level1_f64<P>(raw, out);
-  } else {
+// The interval of the level-LEV entry whose first raw row is at p (rows d = 64*NW apart): all raw loads in flight
+// at once while the entry covers at most 16 rows, else child by child.
+template <int NW, int P, int LEV>
+__device__ __forceinline__ void iv_mem(const __nv_bfloat16* p, uint64_t (&up)[NW], uint64_t (&dn)[NW]) {
+  constexpr int D = 64 * NW;
+  constexpr int R = ipow(P, LEV);
+  if constexpr (R <= 16) {
+    RowW<NW> raw[R];
 #pragma unroll
-    for (int c = 0; c < P; ++c) {
-      double ch[8];
-      tree_from_raw<P, LEV - 1>(raw + c * ipow(P, LEV - 1), ch);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? ch[i] : out[i] + ch[i];
-    }
-  }
-}
-
-template <int D, int P, int LEV>
-__device__ __forceinline__ void tree_sum(const __nv_bfloat16* p, double (&out)[8]) {
-  if constexpr (ipow(P, LEV) <= 16) {
-    // few enough rows to keep all of their loads in flight at once; the sums keep the tree order
-    constexpr int R = ipow(P, LEV);
-    uint4 raw[R];
-#pragma unroll
-    for (int u = 0; u < R; ++u) raw[u] = ld16(p + (int64_t)u * D);
-    tree_from_raw<P, LEV>(raw, out);
-  } else if constexpr (LEV == 1) {
-    uint4 raw[P];
-#pragma unroll
-    for (int u = 0; u < P; ++u) raw[u] = ld16(p + (int64_t)u * D);
-    level1_f64<P>(raw, out);
+    for (int u = 0; u < R; ++u) raw[u] = ld_roww<NW>(p + (int64_t)u * D);
+    iv_regs<NW, P, LEV>(raw, up, dn);
   } else {
     constexpr int CW = ipow(P, LEV - 1);
 #pragma unroll 1
     for (int c = 0; c < P; ++c) {
-      double ch[8];
-      tree_sum<D, P, LEV - 1>(p + (int64_t)c * CW * D, ch);
+      uint64_t cu[NW], cd[NW];
+      iv_mem<NW, P, LEV - 1>(p + (int64_t)c * CW * D, cu, cd);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = (c == 0) ? ch[i] : out[i] + ch[i];
+      for (int i = 0; i < NW; ++i) {
+        up[i] = c == 0 ? cu[i] : add2_up(up[i], cu[i]);
+        dn[i] = c == 0 ? cd[i] : add2_dn(dn[i], cd[i]);
+      }
     }
   }
 }
 
-// Pooled (bf16) value of entry (lev, j) recomputed from the raw rows with the same summation tree as the pool
-// kernel: a level-1 entry whose fp32 chains agree is rounded straight from fp32.
-template <int D, int P>
-__device__ __forceinline__ uint4 pooled_row(const __nv_bfloat16* x0, int lev) {
-  double s[8], val[8];
-  if (lev == 1) {
-    uint4 raw[P];
+// The pooled bf16 values from an interval: true when both copies agree on every value and sum * 2^-(LEV log2 p)
+// is zero or a normal number (then that fp32 product is exact and its bf16 rounding is the definition's).
+template <int NW>
+__device__ __forceinline__ bool iv_finish(const uint64_t (&up)[NW], const uint64_t (&dn)[NW], float scale,
+                                          RowW<NW>& out) {
+  uint32_t diff = 0u;
+  bool normal = true;
 #pragma unroll
-    for (int u = 0; u < P; ++u) raw[u] = ld16(x0 + (int64_t)u * D);
-    float up[8], pv[8];
-    bool fast = level1_f32<P>(raw, up);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      pv[i] = mul_rn(up[i], 1.0f / (float)P);
-      fast &= zero_or_normal(pv[i]);
-    }
-    if (fast)
-      return make_uint4(pack_bf16x2_rn(pv[0], pv[1]), pack_bf16x2_rn(pv[2], pv[3]), pack_bf16x2_rn(pv[4], pv[5]),
-                        pack_bf16x2_rn(pv[6], pv[7]));
-    tree_sum<D, P, 1>(x0, s);
-  } else if (lev == 2) {
-    tree_sum<D, P, 2>(x0, s);
-  } else if (lev == 3) {
-    tree_sum<D, P, 3>(x0, s);
-  } else {
-    tree_sum<D, P, 4>(x0, s);
+  for (int i = 0; i < NW; ++i) {
+    const float u0 = __uint_as_float((uint32_t)up[i]), u1 = __uint_as_float((uint32_t)(up[i] >> 32));
+    const float d0 = __uint_as_float((uint32_t)dn[i]), d1 = __uint_as_float((uint32_t)(dn[i] >> 32));
+    // x - y is zero exactly when x == y (gradual underflow); inf - inf and NaN give NaN, never zero
+    diff |= __float_as_uint(sub_rn(u0, d0)) | __float_as_uint(sub_rn(u1, d1));
+    const float v0 = mul_rn(u0, scale), v1 = mul_rn(u1, scale);
+    normal &= zero_or_normal(v0) & zero_or_normal(v1);
+    out.w[i] = pack_bf16x2_rn(v0, v1);
   }
-  return round_pooled(s, 1.0 / (double)ipow(P, lev), val);
+  return normal && (diff & 0x7FFFFFFFu) == 0u;
 }
 
-// One group per gathered row (b, h, s): copy (level 0), read (pyramid) or recompute (pooled) the row, and store
-// it as fp16, the operand format of the attention kernels (every bf16 value of magnitude in [2^-14, 65504] is
-// exact in fp16; a larger one records LH_ERR_RANGE).
-// Small blocks (kGatherThreads), many per SM: rows cost from one to p^(L-2) raw rows, and a block retires only
-// with its slowest row.
-constexpr int kGatherThreads = 32;
+// The definition's tree in fp64, for lanes whose interval did not close: the raw rows one at a time, level-1
+// sums from the raw values, and every completed entry added into its parent (children left to right from the
+// first).  A real call with the level as an argument: the path is rare, and inlined it would set the register
+// budget of the whole kernel.
+template <int NW, int P>
+__device__ __noinline__ RowW<NW> pooled_f64(const __nv_bfloat16* p, int lev) {
+  constexpr int D = 64 * NW;
+  double acc[LH_MAX_LEVELS][2 * NW];  // acc[l]: running sum of the current level-l entry (l >= 1)
+  int rows = 1;
+  for (int l = 0; l < lev; ++l) rows *= P;
+#pragma unroll 1
+  for (int u = 0; u < rows; ++u) {
+    const RowW<NW> r = ld_roww<NW>(p + (int64_t)u * D);
+    double x[2 * NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      x[2 * i] = f64_of(__uint_as_float(r.w[i] << 16));
+      x[2 * i + 1] = f64_of(__uint_as_float(r.w[i] & 0xFFFF0000u));
+    }
+    int j = u;  // index of the entry just completed one level down
+#pragma unroll 1
+    for (int l = 1; l <= lev; ++l) {
+      const int c = j % P;
+#pragma unroll
+      for (int e = 0; e < 2 * NW; ++e) {
+        const double ch = l == 1 ? x[e] : acc[l - 1][e];
+        acc[l][e] = c == 0 ? ch : acc[l][e] + ch;
+      }
+      if (c != P - 1) break;
+      j /= P;
+    }
+  }
+  double inv_w = 1.0;
+  for (int l = 0; l < lev; ++l) inv_w *= 1.0 / (double)P;  // exact: p is a power of two
+  RowW<NW> out;
+#pragma unroll
+  for (int i = 0; i < NW; ++i)
+    out.w[i] = f64_to_bf16_bits_rne(acc[lev][2 * i] * inv_w) | (f64_to_bf16_bits_rne(acc[lev][2 * i + 1] * inv_w) << 16);
+  return out;
+}
+
+template <int NW, int P, int LEV>
+__device__ __forceinline__ RowW<NW> pooled_lev(const __nv_bfloat16* p) {
+  uint64_t up[NW], dn[NW];
+  iv_mem<NW, P, LEV>(p, up, dn);
+  RowW<NW> out;
+  if (!iv_finish<NW>(up, dn, 1.0f / (float)ipow(P, LEV), out)) out = pooled_f64<NW, P>(p, LEV);
+  return out;
+}
+
+// Pooled (bf16) value of a level-lev entry recomputed from its raw rows, bit-identical to the pool kernel's.
+// Levels above 3 are never recomputed by the layer (it keeps at most five levels and stores the coarsest);
+// they take the fp64 path.
+template <int NW, int P>
+__device__ __forceinline__ RowW<NW> pooled_row(const __nv_bfloat16* p, int lev) {
+  switch (lev) {
+    case 1: return pooled_lev<NW, P, 1>(p);
+    case 2: return pooled_lev<NW, P, 2>(p);
+    case 3: return pooled_lev<NW, P, 3>(p);
+    default: return pooled_f64<NW, P>(p, lev);
+  }
+}
+
+// bf16 -> fp16 (the attention kernels' operand format) and store.  Exact for every bf16 value of magnitude in
+// [2^-14, 65504]; smaller ones round to fp16 subnormals, larger ones set *overflow.
+template <int NW>
+__device__ __forceinline__ void st_f16(__half* p, const RowW<NW>& v, bool& overflow) {
+  uint32_t o[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    const float lo = __uint_as_float(v.w[i] << 16), hi = __uint_as_float(v.w[i] & 0xFFFF0000u);
+    __half2 h = __floats2half2_rn(lo, hi);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+    overflow |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+  }
+  if constexpr (NW == 2)
+    *reinterpret_cast<uint2*>(p) = make_uint2(o[0], o[1]);
+  else
+    *reinterpret_cast<uint32_t*>(p) = o[0];
+}
+
+__device__ __forceinline__ int64_t shfl64(int64_t v, int src) {
+  const int lo = __shfl_sync(0xffffffffu, (int)(uint32_t)v, src);
+  const int hi = __shfl_sync(0xffffffffu, (int)(uint32_t)((uint64_t)v >> 32), src);
+  return (int64_t)(((uint64_t)(uint32_t)hi << 32) | (uint32_t)lo);
+}
+
+// Each warp takes a run of kGatherRun consecutive gathered rows of one job: lane i reads the index of row i (one
+// coalesced load) and works out its source; then, kGatherBatch rows at a time, the warp issues the loads of all
+// copied rows (level 0 from x, stored levels from the pyramid) together, recomputes the pooled rows one by one
+// while those are in flight, and stores everything as fp16.
+constexpr int kGatherWarps = 4;
+constexpr int kGatherRun = 32;
+constexpr int kGatherBatch = 8;
+constexpr int kSrcCopy = 0x100;  // code bit: the row is copied (bit 0: from the pyramid); else code = its level
 
 template <int D, int P>
-__global__ void __launch_bounds__(kGatherThreads, 16) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
-                                                                 LhDims dm) {
-  constexpr int G = D / 8;
+__global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherJobs jobs, const int32_t* __restrict__ idx_g,
+                                                                   LhDims dm) {
+  constexpr int NW = D / 64;
   const GatherJob& job = jobs.job[blockIdx.y];
-  const int lane = threadIdx.x % G;
-  const int64_t row = (int64_t)blockIdx.x * (kGatherThreads / G) + threadIdx.x / G;
-  if (row >= (int64_t)dm.BH * dm.S) return;
-  const int bh = (int)(row / dm.S);
-  const int gid = idx_g[row];
-  int lev = 0;
-#pragma unroll
-  for (int l = 1; l < LH_MAX_LEVELS; ++l)
-    if (l < dm.L && gid >= dm.off[l]) lev = l;
-  const int j = gid - dm.off[lev];
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)dm.BH * dm.S;
+  const int64_t row0 = ((int64_t)blockIdx.x * kGatherWarps + threadIdx.x / 32) * kGatherRun;
+  if (row0 >= rows) return;  // whole warps only
   const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(job.x);
-  uint4 v;
-  if (lev == 0) {
-    v = ld16(x + ((int64_t)bh * dm.N + j) * D + lane * 8);
-  } else if ((job.pyr_mask >> lev) & 1u) {
-    v = ld16(reinterpret_cast<const __nv_bfloat16*>(job.pyr) +
-             ((int64_t)bh * job.pyr_rows + job.row_off[lev] + j) * D + lane * 8);
-  } else {
-    v = pooled_row<D, P>(x + ((int64_t)bh * dm.N + (int64_t)j * dm.wl[lev]) * D + lane * 8, lev);
+  const __nv_bfloat16* pyr = reinterpret_cast<const __nv_bfloat16*>(job.pyr);
+  __half* out = reinterpret_cast<__half*>(job.out);
+
+  int code = -1;  // -1: past the last row
+  int64_t src = 0;  // element offset of the row's first source row
+  if (row0 + lane < rows) {
+    const int64_t row = row0 + lane;
+    const int bh = (int)(row / dm.S);
+    const int gid = idx_g[row];
+    int lev = 0;
+#pragma unroll
+    for (int l = 1; l < LH_MAX_LEVELS; ++l)
+      if (l < dm.L && gid >= dm.off[l]) lev = l;
+    const int j = gid - dm.off[lev];
+    if (lev == 0) {
+      code = kSrcCopy;
+      src = ((int64_t)bh * dm.N + j) * D;
+    } else if ((job.pyr_mask >> lev) & 1u) {
+      code = kSrcCopy | 1;
+      src = ((int64_t)bh * job.pyr_rows + job.row_off[lev] + j) * D;
+    } else {
+      code = lev;
+      src = ((int64_t)bh * dm.N + (int64_t)j * dm.wl[lev]) * D;
+    }
   }
+  const int col = lane * 2 * NW;
   bool overflow = false;
-  const uint4 h = bf16x8_to_f16x8(v, overflow);
+#pragma unroll 1
+  for (int b0 = 0; b0 < kGatherRun && row0 + b0 < rows; b0 += kGatherBatch) {
+    RowW<NW> v[kGatherBatch];
+    int cr[kGatherBatch];
+#pragma unroll
+    for (int r = 0; r < kGatherBatch; ++r) {
+      cr[r] = __shfl_sync(0xffffffffu, code, b0 + r);
+      const int64_t sr = shfl64(src, b0 + r);
+      if (cr[r] >= kSrcCopy) v[r] = ld_roww<NW>(((cr[r] & 1) ? pyr : x) + sr + col);
+    }
+#pragma unroll 1
+    for (int r = 0; r < kGatherBatch; ++r) {
+      const int c = __shfl_sync(0xffffffffu, code, b0 + r);
+      const int64_t sr = shfl64(src, b0 + r);
+      if (c >= 1 && c < kSrcCopy) st_f16<NW>(out + (row0 + b0 + r) * D + col, pooled_row<NW, P>(x + sr + col, c), overflow);
+    }
+#pragma unroll
+    for (int r = 0; r < kGatherBatch; ++r)
+      if (cr[r] >= kSrcCopy) st_f16<NW>(out + (row0 + b0 + r) * D + col, v[r], overflow);
+  }
   if (overflow) set_status(dm.status, LH_ERR_RANGE);
-  st16(reinterpret_cast<__half*>(job.out) + row * D + lane * 8, h);
 }
 
 // Jobs with scores and jobs without run as two launches of the two specialisations (the one without carries no
@@ -437,14 +557,16 @@ int launch_pool_d(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_
 
 template <int D>
 int launch_gather_d(const GatherJobs& jobs, int njobs, const int32_t* idx_g, const LhDims& dm, cudaStream_t st) {
-  constexpr int G = D / 8;
   const int64_t rows = (int64_t)dm.BH * dm.S;
-  const int64_t blocks = (rows + kGatherThreads / G - 1) / (kGatherThreads / G);
+  const int64_t warps = (rows + kGatherRun - 1) / kGatherRun;
+  const int64_t blocks = (warps + kGatherWarps - 1) / kGatherWarps;
+  if (blocks == 0) return LH_OK;
+  if (blocks > 0x7fffffff) return LH_ERR_UNSUPPORTED;
   dim3 grid((unsigned)blocks, njobs);
   switch (dm.p) {
-    case 2: gather_kernel<D, 2><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
-    case 4: gather_kernel<D, 4><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
-    case 8: gather_kernel<D, 8><<<grid, kGatherThreads, 0, st>>>(jobs, idx_g, dm); break;
+    case 2: gather_kernel<D, 2><<<grid, kGatherWarps * 32, 0, st>>>(jobs, idx_g, dm); break;
+    case 4: gather_kernel<D, 4><<<grid, kGatherWarps * 32, 0, st>>>(jobs, idx_g, dm); break;
+    case 8: gather_kernel<D, 8><<<grid, kGatherWarps * 32, 0, st>>>(jobs, idx_g, dm); break;
     default: return LH_ERR_UNSUPPORTED;
   }
   return check_launch();

@@ -50,3 +50,30 @@ def make_scores(B: int, H: int, rows: int, seed: int = 0, device="cpu", ties: bo
         return torch.randint(0, 4, (B, H, rows), generator=g, device=device).to(torch.float32)
     z = torch.randn((B, H, rows), generator=g, device=device, dtype=torch.float32)
     return z * z
+
+
+def make_hard_inputs(B: int, H: int, N: int, d: int, seed: int = 0, device="cpu", emin: int = -140, emax: int = 3):
+    """``(q, k, v)`` bf16 tensors ``[B, H, N, d]`` whose values stress exact summation and the number formats.
+
+    Every value is ``sign * (1 + m/128) * 2^e`` with a random sign, a random 7-bit ``m`` and an exponent ``e``
+    drawn per element from ``[emin, emax]`` in half of the rows, and from a three-wide band at a random height in the
+    other half (so whole pooled entries can be tiny, with sums in the subnormal range); about one value in eight is a
+    zero of either sign.  Values below 2^-126 become bf16 subnormals (or zero) in the final rounding to bf16.  The
+    default range keeps every value below 16, inside the fp16 range of the attention operands."""
+    g = _generator(seed, device)
+    shape = (B, H, N, d)
+    rows = shape[:-1] + (1,)
+
+    def one():
+        sign = torch.randint(0, 2, shape, generator=g, device=device).to(torch.float64) * 2 - 1
+        mant = 1 + torch.randint(0, 128, shape, generator=g, device=device).to(torch.float64) / 128
+        e_elem = torch.randint(emin, emax + 1, shape, generator=g, device=device)
+        e_band = (torch.randint(emin + 2, emax + 1, rows, generator=g, device=device)
+                  - torch.randint(0, 3, shape, generator=g, device=device))
+        banded = torch.rand(rows, generator=g, device=device) < 0.5
+        e = torch.where(banded, e_band, e_elem).to(torch.float64)
+        zero = torch.rand(shape, generator=g, device=device) < 0.125
+        x = sign * torch.where(zero, torch.zeros_like(mant), mant * torch.exp2(e))
+        return x.to(torch.float32).to(torch.bfloat16)
+
+    return one(), one(), one()
