@@ -10,9 +10,12 @@
 // Sentinel key 0 is below every real key.
 //
 // One CTA (8 warps) per (head, level, chunk).  Each warp keeps a running top-M (M = picks rounded up to a power
-// of two) of its share of the chunk in registers, M/32 keys per lane, sorted descending.  A new block of M keys is
+// of two) of its share of the chunk in registers, M/32 keys per lane, sorted descending.  Keys of the warp's
+// blocks that exceed the running M-th largest key are compacted (ballot) into a per-warp shared-memory buffer;
+// a key at or below it can never enter the warp's top M, since M larger-or-equal keys are already held and keys
+// are unique.  When the next block's candidates would overflow the buffer, and at the end, the buffer is
 // bitonic-sorted ascending (register compare-exchange for partners in the same lane, warp shuffles otherwise);
-// the element-wise maximum of the descending running list and the ascending block is a bitonic sequence that
+// the element-wise maximum of the descending running list and the ascending buffer is a bitonic sequence that
 // holds the top M of both, which one bitonic merge sorts descending again.  The eight warp lists are merged the
 // same way through shared memory.
 #include "internal.h"
@@ -30,6 +33,13 @@ __device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int mask) {
   uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
   lo = __shfl_xor_sync(0xffffffffu, lo, mask);
   hi = __shfl_xor_sync(0xffffffffu, hi, mask);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl_idx64(uint64_t v, int src) {
+  uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
+  lo = __shfl_sync(0xffffffffu, lo, src);
+  hi = __shfl_sync(0xffffffffu, hi, src);
   return ((uint64_t)hi << 32) | lo;
 }
 
@@ -103,21 +113,46 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   uint64_t top[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) top[r] = 0;
-  const int nblocks = (nc + M - 1) / M;
-  for (int b = warp; b < nblocks; b += 8) {
+  uint64_t thr = 0;  // the running M-th largest key (0: fewer than M keys so far)
+  uint64_t* buf = s_top[warp];  // candidate buffer (the warp's merge slot is free until the end)
+  int cnt = 0;                  // keys in the buffer (warp-uniform)
+  auto flush = [&]() {          // fold the buffer into the running list
+    __syncwarp();
     uint64_t key[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int e = b * M + lane * R + r;
-      key[r] = e < nc ? make_key(sc[e], (uint32_t)(c * nc + e)) : 0ull;
-    }
+    for (int r = 0; r < R; ++r) key[r] = lane * R + r < cnt ? buf[lane * R + r] : 0ull;
+    __syncwarp();
     bitonic_sort_asc<R, 2>(key, lane);
 #pragma unroll
     for (int r = 0; r < R; ++r) key[r] = top[r] > key[r] ? top[r] : key[r];
     merge_desc<R, M / 2>(key, lane);
 #pragma unroll
     for (int r = 0; r < R; ++r) top[r] = key[r];
+    thr = shfl_idx64(top[R - 1], 31);
+    cnt = 0;
+  };
+  const unsigned lt = (1u << lane) - 1u;  // lanes below this one
+  const int nblocks = (nc + M - 1) / M;
+  for (int b = warp; b < nblocks; b += 8) {
+    uint64_t key[R];
+    int nb = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = b * M + r * 32 + lane;  // coalesced: element r*32 + lane of the block
+      key[r] = e < nc ? make_key(sc[e], (uint32_t)(c * nc + e)) : 0ull;
+      nb += __popc(__ballot_sync(0xffffffffu, key[r] > thr));
+    }
+    if (cnt + nb > M) flush();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const bool keep = key[r] > thr;
+      const unsigned vote = __ballot_sync(0xffffffffu, keep);
+      if (keep) buf[cnt + __popc(vote & lt)] = key[r];
+      cnt += __popc(vote);
+    }
   }
+  if (cnt > 0) flush();
+  __syncwarp();
 #pragma unroll
   for (int r = 0; r < R; ++r) s_top[warp][lane * R + r] = top[r];
   __syncthreads();
