@@ -358,20 +358,17 @@ def main():
     tokens = whole_job_tokens(w, world)
     value = tokens / (ms / 1e3)
 
-    # end to end through the C ABI with host buffers: H2D of the step's inputs, the step, D2H of its outputs
+    # end to end through the C ABI with host buffers (lh_step_host): every step copies its inputs from page-locked
+    # host memory and its outputs back, chunk by chunk of heads, the two copy directions and the compute overlapped
     e2e = None
     if not args.no_e2e:
         host_in = [t.cpu().pin_memory() for t in (q, k, v, dout)]
         host_out = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
-        dev_in = (q, k, v, dout)
-        dev_out = (o, dq, dk, dv)
+        hc = lh.default_heads_per_chunk(P)
+        dev_buf = torch.empty(lh.lh_step_host_bytes(P, hc), dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            for h, d_ in zip(host_in, dev_in):
-                d_.copy_(h, non_blocking=True)
-            step()
-            for h, d_ in zip(host_out, dev_out):
-                h.copy_(d_, non_blocking=True)
+            lh.lh_step_host(P, *host_in, *host_out, heads_per_chunk=hc, dev_buf=dev_buf, device=dev)
 
         e2e_step()
         torch.cuda.synchronize(dev)
@@ -390,7 +387,8 @@ def main():
         nbytes = sum(t.numel() * t.element_size() for t in host_in)
         obytes = sum(t.numel() * t.element_size() for t in host_out)
         e2e = {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
-               "d2h_bytes_per_step": obytes, "ms_per_step": ms_e2e, "steps": n_e2e}
+               "d2h_bytes_per_step": obytes, "ms_per_step": ms_e2e, "steps": n_e2e,
+               "pipeline": f"lh_step_host, {w['B'] * (w['H'] // hc)} chunks of {hc} heads"}
 
     peaks = load_peaks()
     work, S = kernel_work(w)

@@ -69,6 +69,9 @@ _SIGS = {
     "lh_score_topk_static": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
     "lh_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "lh_profile_read": (ctypes.c_int, [ctypes.POINTER(LhKernelTime), ctypes.c_int]),
+    "lh_step_host_bytes": (ctypes.c_size_t, [_P, ctypes.c_int]),
+    "lh_step_host": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_size_t, _vp,
+                                    _vp, _vp]),
 }
 
 
@@ -310,6 +313,66 @@ def lh_backward(P: Params, dout, ctx, dq=None, dk=None, dv=None, ws=None):
                           ws.numel(), _stream(dev))
     _check(rc, "lh_backward")
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------------------------------------------------
+# Host-resident step (host tensors in, host tensors out; the copies are pipelined inside the library)
+# ------------------------------------------------------------------------------------------------------------
+
+_copy_streams: dict = {}
+
+
+def default_heads_per_chunk(P: Params) -> int:
+    """The largest divisor of H that still gives at least eight chunks per batch row (one head when H < 8)."""
+    best = 1
+    for hc in range(1, P.H + 1):
+        if P.H % hc == 0 and P.H // hc >= 8:
+            best = hc
+    return best
+
+
+def lh_step_host_bytes(P: Params, heads_per_chunk: int) -> int:
+    return _lib.lh_step_host_bytes(ctypes.byref(P.c()), int(heads_per_chunk))
+
+
+def _host_bf16(t, shape, name):
+    _typed(t, shape, name, torch.bfloat16)
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous host (CPU) tensor")
+    return t.data_ptr()
+
+
+def lh_step_host(P: Params, q, k, v, dout, o=None, dq=None, dk=None, dv=None, heads_per_chunk=None, dev_buf=None,
+                 device=None):
+    """lh_forward + lh_backward on HOST bf16 tensors [B,H,N,d] (page-locked for overlap), returning host (o, dq, dk,
+    dv).  Runs on `device` (default: the current CUDA device): the compute on its current stream, the copies on two
+    streams of this module; returns once everything is enqueued (synchronise the current stream before reading the
+    outputs)."""
+    _valid(P, "lh_step_host")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    hc = default_heads_per_chunk(P) if heads_per_chunk is None else int(heads_per_chunk)
+    shape = (P.B, P.H, P.N, P.d)
+    ins = [_host_bf16(t, shape, n) for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"))]
+    outs = []
+    for t, n in ((o, "o"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        outs.append(torch.empty(shape, dtype=torch.bfloat16, pin_memory=True) if t is None else t)
+    out_ptrs = [_host_bf16(t, shape, n) for t, n in zip(outs, ("o", "dq", "dk", "dv"))]
+    need = lh_step_host_bytes(P, hc)
+    if need == 0:
+        raise LighthouseError(LH_ERR_INVALID_ARG, "lh_step_host_bytes")
+    if dev_buf is None:
+        dev_buf = torch.empty(need, dtype=torch.uint8, device=dev)
+    if dev_buf.device != dev:
+        raise ValueError("dev_buf must live on the step's device")
+    key = dev.index
+    if key not in _copy_streams:
+        _copy_streams[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    h2d, d2h = _copy_streams[key]
+    with torch.cuda.device(dev):
+        rc = _lib.lh_step_host(ctypes.byref(P.c()), *ins, *out_ptrs, hc, _ptr(dev_buf), dev_buf.numel(),
+                               torch.cuda.current_stream(dev).cuda_stream, h2d.cuda_stream, d2h.cuda_stream)
+    _check(rc, "lh_step_host")
+    return tuple(outs)
 
 
 def lh_scatter_bwd(P: Params, dout, idx_g, dog=None):

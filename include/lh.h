@@ -216,6 +216,34 @@ int lh_profile_read(lh_kernel_time_t* out, int max_entries);
 int lh_score_topk_static(const lh_params* P, const void* k, const float* scores_in, float* scores_out,
                          int32_t* idx_g, int32_t* slot, void* stream);
 
+/* ---- host-resident step ------------------------------------------------------------------------------ */
+
+/* Device bytes lh_step_host needs with chunks of `heads_per_chunk` heads (0 if P is invalid or heads_per_chunk
+ * does not divide H): two chunks' eight tensors, one chunk's ctx and one chunk's workspace. */
+size_t lh_step_host_bytes(const lh_params* P, int heads_per_chunk);
+
+/* The pages have no counterpart to this entry point: it serves callers whose tensors live in host memory.
+ *
+ * One lh_forward + lh_backward on HOST tensors: q, k, v, dout (bf16 [B,H,N,d], read) -> o, dq, dk, dv (bf16
+ * [B,H,N,d], written); results equal those of the device entry points on the same data (each head is computed
+ * alone, exactly as in a call over all heads).  Heads are independent through the whole layer, so the work runs in
+ * chunks of heads_per_chunk consecutive heads of one batch row (heads_per_chunk must divide H): chunk g's
+ * host-to-device copies (on h2d_stream), its forward and backward (on stream) and its device-to-host copies (on
+ * d2h_stream) overlap with the neighbouring chunks'.  Host buffers should be page-locked: pageable memory makes the
+ * copies synchronous and serialises the pipeline (results are the same).  The three streams should be distinct
+ * for the overlap (any of them may be NULL, the legacy default stream, at the cost of it).
+ * dev: caller's device buffer of at least lh_step_host_bytes(P, heads_per_chunk) bytes, 256-byte aligned; it is
+ * scratch only (nothing is kept in it between calls).  Everything is enqueued: the copies start after the work
+ * already on `stream`, and `stream` is ordered after the last device-to-host copy, so synchronising `stream`
+ * makes o, dq, dk, dv valid on the host.  Errors: LH_ERR_INVALID_ARG (sizes, heads_per_chunk, NULL or misaligned
+ * pointers), LH_ERR_WORKSPACE (dev_bytes too small), LH_ERR_CUDA (a copy, event or launch failed), or the error
+ * of lh_forward / lh_backward; a failure mid-way leaves the earlier chunks enqueued.  The pipeline's events are
+ * created on the first call on each device and reused, so concurrent calls on one device from several host
+ * threads must be serialised by the caller. */
+int lh_step_host(const lh_params* P, const void* q, const void* k, const void* v, const void* dout, void* o, void* dq,
+                 void* dk, void* dv, int heads_per_chunk, void* dev, size_t dev_bytes, void* stream, void* h2d_stream,
+                 void* d2h_stream);
+
 /* ---- status ------------------------------------------------------------------------------------------ */
 
 /* Synchronises `stream`, returns the first device-side error recorded since the last call (LH_OK if none)

@@ -103,3 +103,31 @@ def test_error_strings(lh):
     for code in range(7):
         assert lh.error_string(code)
     assert lh.error_string(99) == "unknown status"
+
+
+def test_step_host_bytes_and_argument_errors(lh):
+    """lh_step_host sizing and the errors it returns on the host, before any CUDA call."""
+    P = lh.Params(2, 4, 4096, 64, 3, 4, 256, 8)
+    Pc = lh.Params(1, 2, 4096, 64, 3, 4, 256, 8)
+    tensor = 2 * 4096 * 64 * 2  # one chunk tensor of two heads, bf16
+    need = lh.lh_step_host_bytes(P, 2)
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert need == 2 * 8 * rnd(tensor) + rnd(lh.lh_ctx_bytes(Pc)) + rnd(lh.lh_workspace_bytes(Pc))
+    assert lh.lh_step_host_bytes(P, 3) == 0  # does not divide H
+    assert lh.lh_step_host_bytes(P, 0) == 0
+    bad = lh.Params(1, 2, 4100, 64, 3, 4, 256, 8)  # p^(L-1) = 16 does not divide N
+    assert lh.lh_validate(bad) != 0 and lh.lh_step_host_bytes(bad, 1) == 0
+    assert lh.default_heads_per_chunk(lh.Params(1, 16, 524288, 128, 4, 4, 4096, 32)) == 2
+    assert lh.default_heads_per_chunk(lh.Params(1, 2, 4096, 64, 3, 4, 256, 8)) == 1
+
+    lib = lh.library()
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.addressof(buf)
+    c = P.c()
+    call = lambda hc, dev, nbytes, ptr=p: lib.lh_step_host(ctypes.byref(c), ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, hc,
+                                                           dev, nbytes, None, None, None)
+    assert call(3, 256, 1 << 40) == lh.LH_ERR_INVALID_ARG           # heads_per_chunk does not divide H
+    assert call(2, None, 1 << 40) == lh.LH_ERR_INVALID_ARG          # no device buffer
+    assert call(2, 256 + 16, 1 << 40) == lh.LH_ERR_INVALID_ARG      # misaligned device buffer
+    assert call(2, 256, need - 1) == lh.LH_ERR_WORKSPACE            # device buffer too small
+    assert call(2, 256, 1 << 40, ptr=None) == lh.LH_ERR_INVALID_ARG  # NULL host tensor
