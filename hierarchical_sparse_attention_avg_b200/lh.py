@@ -323,10 +323,12 @@ _copy_streams: dict = {}
 
 
 def default_heads_per_chunk(P: Params) -> int:
-    """The largest divisor of H that still gives at least eight chunks per batch row (one head when H < 8)."""
+    """The largest divisor of H that still gives at least sixteen chunks per batch row (one head when H < 16): the
+    first chunk's host-to-device copy and the last chunk's device-to-host copy are not overlapped, so small chunks
+    pay less for them."""
     best = 1
     for hc in range(1, P.H + 1):
-        if P.H % hc == 0 and P.H // hc >= 8:
+        if P.H % hc == 0 and P.H // hc >= 16:
             best = hc
     return best
 

@@ -117,7 +117,8 @@ def test_step_host_bytes_and_argument_errors(lh):
     assert lh.lh_step_host_bytes(P, 0) == 0
     bad = lh.Params(1, 2, 4100, 64, 3, 4, 256, 8)  # p^(L-1) = 16 does not divide N
     assert lh.lh_validate(bad) != 0 and lh.lh_step_host_bytes(bad, 1) == 0
-    assert lh.default_heads_per_chunk(lh.Params(1, 16, 524288, 128, 4, 4, 4096, 32)) == 2
+    assert lh.default_heads_per_chunk(lh.Params(1, 16, 524288, 128, 4, 4, 4096, 32)) == 1
+    assert lh.default_heads_per_chunk(lh.Params(1, 64, 4096, 64, 3, 4, 256, 8)) == 4
     assert lh.default_heads_per_chunk(lh.Params(1, 2, 4096, 64, 3, 4, 256, 8)) == 1
 
     lib = lh.library()
