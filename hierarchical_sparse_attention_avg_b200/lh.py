@@ -349,7 +349,7 @@ def lh_step_host(P: Params, q, k, v, dout, o=None, dq=None, dk=None, dv=None, he
     """lh_forward + lh_backward on HOST bf16 tensors [B,H,N,d] (page-locked for overlap), returning host (o, dq, dk,
     dv).  Runs on `device` (default: the current CUDA device): the compute on its current stream, the copies on two
     streams of this module; returns once everything is enqueued (synchronise the current stream before reading the
-    outputs)."""
+    outputs, and keep the input tensors alive until then: the library copies from them asynchronously)."""
     _valid(P, "lh_step_host")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     hc = default_heads_per_chunk(P) if heads_per_chunk is None else int(heads_per_chunk)
