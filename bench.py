@@ -36,6 +36,8 @@ WORKLOADS = {
     # variant parameters: the recipe's L=3, k=1536, and the ablation grid's L in {3, 4}, k in {1536, 2048} at 98K
     "recipe98K": dict(B=1, H=16, N=98304, d=64, L=3, p=4, k=1536, C=16),
     "ablation98K_L4k1536": dict(B=1, H=16, N=98304, d=64, L=4, p=4, k=1536, C=16),
+    # the children-expansion reading at the pages' size example (S = 65,536 at N = 2^20)
+    "stress1M_expand": dict(B=1, H=8, N=1048576, d=128, L=4, p=4, k=4096, C=32, expand=True),
 }
 DEFAULT_WORKLOAD = "long512K"
 METRIC = "Lighthouse fwd+bwd tokens/s at N=512K; HBM GB/s and attention TFLOP/s vs peak"
@@ -54,18 +56,27 @@ def load_peaks():
 def kernel_work(w: dict) -> dict:
     """Algorithmic bytes (HBM-bound kernels) or FLOPs (attention) of ONE launch of each kernel, all heads."""
     B, H, N, d, L, p, k = w["B"], w["H"], w["N"], w["d"], w["L"], w["p"], w["k"]
+    expand = w.get("expand", False)
     BH = B * H
     Nl = [N // p ** lev for lev in range(L)]
-    kl = [min(k, Nl[lev]) if lev < L - 1 else Nl[lev] for lev in range(L)]
+    if expand:  # level lev keeps the p children of the picks of level lev + 1
+        kl = [p * min(k, Nl[lev + 1]) if lev < L - 1 else Nl[lev] for lev in range(L)]
+        ranked = [lev + 1 for lev in range(L - 1) if kl[lev] < Nl[lev]]
+        Rs = sum(Nl[1:])
+    else:
+        kl = [min(k, Nl[lev]) if lev < L - 1 else Nl[lev] for lev in range(L)]
+        ranked = [lev for lev in range(L - 1) if kl[lev] < Nl[lev]]
+        Rs = sum(Nl[:-1])
     S = sum(kl)
-    R, Rs = sum(Nl), sum(Nl[:-1])
+    R = sum(Nl)
     row = d * 2
     # rows of the raw input that selected entries below the coarsest level cover (read by the gather)
     gather_src = sum(kl[lev] * p ** lev for lev in range(L - 1)) + Nl[-1]
-    partial = sum(Nl[lev] for lev in range(L - 1) if kl[lev] < Nl[lev])
+    partial = sum(Nl[lev] for lev in ranked)  # scores read by the top-K
+    slots_init = sum(Nl[lev] for lev in range(L - 1) if kl[lev] < Nl[lev])
     return {
         "pool_score": ("hbm", BH * (3 * N * row + 3 * Nl[-1] * row + Rs * 4)),
-        "topk": ("hbm", BH * (partial * 4 * 2 + sum(kl[:-1]) * 4)),
+        "topk": ("hbm", BH * (partial * 4 + slots_init * 4 + sum(kl[:-1]) * 4)),
         "order": ("hbm", BH * (S * 4 * 2 + sum(kl[:-1]) * 4)),
         "gather": ("hbm", BH * 3 * (gather_src + S) * row),
         "attn_fwd": ("tensor", 2.0 * S * S * d * BH),
@@ -78,8 +89,22 @@ def kernel_work(w: dict) -> dict:
     }, S
 
 
-# DRAM traffic per launch from a one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), recorded in
-# profiles/dram_traffic.txt with a digest of the kernel's sources; reported only while the sources still match.
+def kernel_bytes(w: dict) -> dict:
+    """Algorithmic DRAM bytes of ONE launch of each kernel (all heads): the HBM-bound kernels' bytes as in
+    kernel_work, and for the attention kernels the unique bytes of their operands and outputs (fp16 gathered rows,
+    fp32 outputs and accumulators, per-row statistics).  Used to scale a DRAM-traffic capture taken on a small
+    workload to another workload of the same kernel."""
+    work, S = kernel_work(w)
+    BH, d = w["B"] * w["H"], w["d"]
+    out = {n: amt for n, (bound, amt) in work.items() if bound == "hbm"}
+    out["attn_fwd"] = BH * S * (3 * d * 2 + d * 4 + 4)
+    out["attn_bwd"] = BH * S * (4 * d * 2 + 2 * 4 + 2 * d * 4 + 2 * d * 4)
+    return out
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one-kernel ncu captures on a small
+# workload, recorded in profiles/dram_traffic.txt with a digest of the kernel's sources; reported (scaled to the
+# bench's workload by the ratio of algorithmic bytes) only while the sources still match.
 TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic.txt")
 CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "hierarchical_sparse_attention_avg_b200", "csrc")
 KERNEL_SOURCES = {"attn_bwd": "attn_bwd.cu", "attn_fwd": "attn_fwd.cu", "pool_score": "pool_gather.cu",
@@ -92,23 +117,29 @@ def source_digest(kernel: str) -> str:
     import hashlib
 
     h = hashlib.sha256()
-    for f in (KERNEL_SOURCES.get(kernel, ""), "lh_common.cuh", "internal.h", "api.cu"):
+    for f in (KERNEL_SOURCES.get(kernel, ""), "lh_common.cuh", "internal.h"):
         path = os.path.join(CSRC, f)
         if f and os.path.exists(path):
             h.update(open(path, "rb").read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, workload: str):
-    """Bytes per launch (read + write) of `kernel` at `workload`, or None when not captured for these sources."""
+def measured_traffic(kernel: str, w: dict):
+    """(bytes per launch at workload w, capture workload) for `kernel`, or (None, None) when no capture matches the
+    current sources.  A capture on another workload is scaled by the ratio of the kernel's algorithmic bytes."""
     if not os.path.exists(TRAFFIC_FILE):
-        return None
+        return None, None
     for line in open(TRAFFIC_FILE):
         f = line.split()
-        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
-            if f[4] == source_digest(kernel):
-                return int(f[2]) + int(f[3])
-    return None
+        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] in WORKLOADS:
+            if f[4] != source_digest(kernel):
+                continue
+            got = int(f[2]) + int(f[3])
+            if WORKLOADS[f[1]] == w:
+                return got, f[1]
+            ratio = kernel_bytes(w)[kernel] / kernel_bytes(WORKLOADS[f[1]])[kernel]
+            return int(round(got * ratio)), f[1]
+    return None, None
 
 
 class NvmlClockSampler:
@@ -239,16 +270,26 @@ def whole_job_tokens(w: dict, world: int) -> int:
     return w["B"] * w["N"] * world
 
 
+def oracle_unavailable(w: dict):
+    """Why the oracle cannot time a head of workload w on the host, or None.  It holds several S x S float64
+    matrices (8 GB each at S = 32K)."""
+    S = kernel_work(w)[1]
+    return f"the oracle's S x S attention matrices at S = {S} exceed host memory" if S > 32768 else None
+
+
 def cpu_baseline(w: dict, seed: int = 0) -> dict:
     """The CPU oracle timed on one head of the workload (forward + backward), scaled to tokens/s of the whole
     workload (heads are independent, so the time of all B*H heads is B*H times one head's)."""
     from oracle import lighthouse as O
     from hierarchical_sparse_attention_avg_b200.inputs import make_inputs
 
+    why = oracle_unavailable(w)
+    if why:
+        return {"unavailable": why, "kind": "oracle"}
     q, k, v, dout = make_inputs(1, 1, w["N"], w["d"], seed=seed, device="cpu")
     f = lambda t: t[0, 0].float().numpy().astype(np.float64)
     qf, kf, vf, df = f(q), f(k), f(v), f(dout)
-    P = O.Params(1, 1, w["N"], w["d"], w["L"], w["p"], w["k"], w["C"])
+    P = O.Params(1, 1, w["N"], w["d"], w["L"], w["p"], w["k"], w["C"], w.get("expand", False))
     t0 = time.perf_counter()
     fwd = O.forward_head(qf, kf, vf, P)
     O.backward_head(df, fwd, P)
@@ -273,27 +314,35 @@ def w_name(w):
 
 
 def run_reference(args, w):
+    """The oracle as the reference arm: W warm-up steps and K timed steps, each one head of the workload
+    (forward + backward) on the host cores; tokens/s of that sample.  Rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    for _ in range(min(args.warmup, 1)):
+    why = oracle_unavailable(w)
+    if why:
+        print(json.dumps({"impl": "reference", "unavailable": why}), flush=True)
+        return
+    for _ in range(max(args.warmup, 0)):
         cpu_baseline(w)
     times = [cpu_baseline(w)["seconds"] for _ in range(args.steps)]
     heads = w["B"] * w["H"]
     sec = sum(times) / len(times)
-    value = w["B"] * w["N"] / (sec * heads)
+    value = w["B"] * w["N"] / (sec * heads)  # the workload's tokens over the time all its heads take
     try:
         from threadpoolctl import threadpool_info
 
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = 1
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
-            "warmup": min(args.warmup, 1), "ms_per_step": sec * 1e3 * heads, "higher_is_better": True,
+    sample = f"one head of {heads} per step (forward+backward; heads are independent)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w_name(w), **w, "sample": "one head per step, scaled by B*H"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"one head of {heads} per step (forward+backward), scaled by {heads}"},
+            "config": {"workload": w_name(w), **w, "sample": sample},
+            "scaled_to_all_heads": {"ms_per_step": sec * 1e3 * heads,
+                                    "note": f"one head's time x {heads} heads: the time the whole step would take"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -398,19 +447,29 @@ def main():
         bound, amount = work.get(name, ("hbm", 0))
         per_ms = kms / launches
         if bound == "tensor":
+            # timed inside a step of milliseconds at full SM clock: the burst GEMM peak applies (the sustained
+            # figure, a seconds-long GEMM loop at the power cap's lower clock, is reported beside it)
             ach = amount / (per_ms / 1e3) / 1e12
             kernels[name] = {"launches": launches, "ms": per_ms, "share": kms / total_kernel_ms, "bound": "tensor",
-                             "achieved": ach, "unit": "TFLOP/s", "frac": ach / peaks["bf16_sust"]}
+                             "achieved": ach, "unit": "TFLOP/s", "frac": ach / peaks["bf16"],
+                             "frac_sustained": ach / peaks["bf16_sust"]}
         else:
             ach = amount / (per_ms / 1e3) / 1e9
             kernels[name] = {"launches": launches, "ms": per_ms, "share": kms / total_kernel_ms, "bound": "hbm",
                              "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm"]}
     top = max(kernels.items(), key=lambda kv: kv[1]["share"])
     tname, tk = top
+    traffic, traffic_src = measured_traffic(tname, w)
     roofline = {"kernel": tname, "bound": tk["bound"], "achieved": tk["achieved"],
-                "peak": peaks["bf16_sust"] if tk["bound"] == "tensor" else peaks["hbm"], "unit": tk["unit"],
-                "frac": tk["frac"], "traffic": measured_traffic(tname, args.workload),
-                "peak_source": f"{peaks['src']} ({'bf16 sustained' if tk['bound'] == 'tensor' else 'HBM copy'})"}
+                "peak": peaks["bf16"] if tk["bound"] == "tensor" else peaks["hbm"], "unit": tk["unit"],
+                "frac": tk["frac"], "traffic": traffic,
+                "peak_source": f"{peaks['src']} ({'bf16 burst' if tk['bound'] == 'tensor' else 'HBM copy'})"}
+    if tk["bound"] == "tensor":
+        roofline["frac_sustained"] = tk["frac_sustained"]
+    if traffic_src is not None:
+        roofline["traffic_source"] = (f"ncu one-kernel capture on {traffic_src}" +
+                                      ("" if traffic_src == args.workload else
+                                       f", scaled by the kernel's algorithmic bytes to {args.workload}"))
     gpu_launches = sum(v_[0] for v_ in prof.values())
 
     if rank == 0:

@@ -9,7 +9,8 @@
 
 namespace lh {
 
-__device__ int g_lh_status = 0;
+// Per-device status word and wait limit (see LhDeviceState).
+__device__ LhDeviceState g_lh_state = {0, 0, kWaitLimitNs};
 
 namespace {
 
@@ -21,7 +22,7 @@ int make_dims(const lh_params* P, LhDims* dm) {
   if (!P) return LH_ERR_INVALID_ARG;
   memset(dm, 0, sizeof(*dm));
   if (P->B < 1 || P->H < 1 || P->N < 1 || P->d < 1 || P->L < 1 || P->p < 2 || P->k < 1 || P->C < 1 ||
-      P->flags != 0 || P->L > LH_MAX_LEVELS)
+      (P->flags & ~LH_EXPAND_CHILDREN) != 0 || P->L > LH_MAX_LEVELS)
     return LH_ERR_INVALID_ARG;
   int64_t w = 1;
   for (int l = 1; l < P->L; ++l) {
@@ -29,9 +30,11 @@ int make_dims(const lh_params* P, LhDims* dm) {
     if (w > P->N) return LH_ERR_INVALID_ARG;
   }
   if (P->N % w) return LH_ERR_INVALID_ARG;
+  const bool expand = (P->flags & LH_EXPAND_CHILDREN) != 0;
   dm->B = P->B; dm->H = P->H; dm->N = P->N; dm->d = P->d; dm->L = P->L; dm->p = P->p; dm->k = P->k; dm->C = P->C;
+  dm->expand = expand ? 1 : 0;
   const int64_t BH = (int64_t)P->B * P->H;
-  int64_t S = 0, R = 0, Rs = 0, Rp = 0;
+  int64_t S = 0, R = 0, Rs = 0, Rp = 0, Ksel = 0;
   int nPartial = 0;
   int64_t wl = 1;
   for (int l = 0; l < P->L; ++l) {
@@ -42,18 +45,26 @@ int make_dims(const lh_params* P, LhDims* dm) {
     while ((int64_t(1) << dm->wlog[l]) < wl) ++dm->wlog[l];  // exact log2 when p is a power of two
     dm->off[l] = (int)R;
     if (l >= 1) dm->poff[l] = (int)Rp;
+    // the level whose scores pick level l's entries: l itself, or its parent level with expand
+    const int64_t n_rank = expand ? n / P->p : n;
     int64_t kl = n;
-    if (l <= P->L - 2 && P->k < n) {
-      if (n % P->C || P->k % P->C) return LH_ERR_INVALID_ARG;
-      kl = P->k;
+    if (l <= P->L - 2 && P->k < n_rank) {
+      if (n_rank % P->C || P->k % P->C) return LH_ERR_INVALID_ARG;
+      kl = expand ? (int64_t)P->k * P->p : P->k;
       if (l != nPartial) return LH_ERR_INVALID_ARG;  // unreachable: level sizes decrease
-      dm->seloff[l] = nPartial * P->k;
+      dm->seloff[l] = (int)Ksel;
+      Ksel += kl;
       ++nPartial;
     }
     dm->kl[l] = (int)kl;
     S += kl;
     R += n;
-    if (l <= P->L - 2) Rs += n;
+    const bool scored = expand ? l >= 1 : l <= P->L - 2;
+    if (scored) {
+      dm->score_mask |= 1u << l;
+      dm->soff[l] = (int)Rs;
+      Rs += n;
+    }
     if (l >= 1) Rp += n;
     wl *= P->p;
   }
@@ -63,13 +74,13 @@ int make_dims(const lh_params* P, LhDims* dm) {
   dm->Rs = (int)Rs;
   dm->Rp = (int)Rp;
   dm->nPartial = nPartial;
-  dm->Ksel = nPartial * P->k;
+  dm->Ksel = (int)Ksel;
   // what the kernels are built for
   if (P->d != 64 && P->d != 128) return LH_ERR_UNSUPPORTED;
   if (P->p != 2 && P->p != 4 && P->p != 8) return LH_ERR_UNSUPPORTED;
   if (P->L > kMaxL || w > 512) return LH_ERR_UNSUPPORTED;
   if (nPartial > 0 && P->k / P->C > 512) return LH_ERR_UNSUPPORTED;
-  if (BH > 65535 || R > INT32_MAX / 2) return LH_ERR_UNSUPPORTED;
+  if (BH > 65535 || R > INT32_MAX / 2 || S > INT32_MAX / 2) return LH_ERR_UNSUPPORTED;
   return LH_OK;
 }
 
@@ -133,8 +144,8 @@ int status_ptr(int** out) {
   std::lock_guard<std::mutex> g(mu);
   if (!cache[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_lh_status) != cudaSuccess) return LH_ERR_CUDA;
-    cache[dev] = static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_lh_state) != cudaSuccess) return LH_ERR_CUDA;
+    cache[dev] = &static_cast<LhDeviceState*>(p)->status;
   }
   *out = cache[dev];
   return LH_OK;
@@ -479,6 +490,17 @@ int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void
   LH_TRY(launch_absmax(dog, amax, dm, st));
   LH_TRY(launch_bwd_prep(dog, og, amax, wsb + w.dog16, dvec, dinv, dqg, dm, st));
   return launch_attn_bwd(qg, kg, vg, wsb + w.dog16, lse, dvec, dinv, dqg, dkg, dvg, dm, st);
+}
+
+int lh_set_wait_limit_ns(uint64_t ns) {
+  int* p = nullptr;
+  if (status_ptr(&p)) return LH_ERR_CUDA;
+  const unsigned long long v = ns ? (unsigned long long)ns : (unsigned long long)kWaitLimitNs;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LH_ERR_CUDA;
+  if (cudaMemcpy(&reinterpret_cast<LhDeviceState*>(p)->wait_limit_ns, &v, sizeof(v), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return LH_ERR_CUDA;
+  return LH_OK;
 }
 
 int lh_get_status(void* stream) {

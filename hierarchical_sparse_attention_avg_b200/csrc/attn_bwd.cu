@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
-  __shared__ int s_abort;
+  __shared__ WaitCtl s_wait;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const float inv_scale = dinv[bh];
 
   if (threadIdx.x == 0) {
-    s_abort = 0;
+    wait_ctl_init(&s_wait, status);
     mbar_init(bar(Lay::B_KV), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(Lay::B_QF + s), 1);
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int it = 0; it < nit && ok; ++it) {
         const int s = it % kStages;
-        if (it >= kStages) ok = mbar_wait(bar(Lay::B_QE + s), ((it / kStages) - 1) & 1, &s_abort, status);
+        if (it >= kStages) ok = mbar_wait(bar(Lay::B_QE + s), ((it / kStages) - 1) & 1, &s_wait, status);
         if (!ok) break;
         const int row = (i0 + it) * kQTile;
         mbar_arrive_expect_tx(bar(Lay::B_QF + s), 2 * Lay::QT);
@@ -144,10 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_f32acc(kFmtF16, 128, kQTile, 0, 0);   // K-major x K-major
       constexpr uint32_t idesc_acc = idesc_f32acc(kFmtF16, 128, D, 0, 1);      // K-major x MN-major
       constexpr uint32_t idesc_dq = idesc_f32acc(kFmtF16, 128, kQTile, 1, 1);  // MN-major x MN-major
-      bool ok = mbar_wait(bar(Lay::B_KV), 0, &s_abort, status);
+      bool ok = mbar_wait(bar(Lay::B_KV), 0, &s_wait, status);
       auto products = [&](int jt) {  // dV, dK, dQ^T of sub-tile jt
         const int b = jt & 1, s = jt % kStages;
-        if (!mbar_wait(bar(Lay::B_DSF + b), (jt >> 1) & 1, &s_abort, status)) return false;
+        if (!mbar_wait(bar(Lay::B_DSF + b), (jt >> 1) & 1, &s_wait, status)) return false;
         tc_fence_after();
         const uint32_t sDS = sb + Lay::DS + b * Lay::PT;
         const uint32_t sQ = sb + Lay::Q + s * Lay::QT, sDO = sb + Lay::DO + s * Lay::QT;
@@ -169,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int it = 0; it < nit && ok; ++it) {
         const int b = it & 1, s = it % kStages;
-        ok = mbar_wait(bar(Lay::B_QF + s), (it / kStages) & 1, &s_abort, status);
+        ok = mbar_wait(bar(Lay::B_QF + s), (it / kStages) & 1, &s_wait, status);
         // buffer pair b: its dQ^T of sub-tile it-2 has been read out of tensor memory
-        if (ok && it >= 2) ok = mbar_wait(bar(Lay::B_DQF + b), ((it >> 1) - 1) & 1, &s_abort, status);
+        if (ok && it >= 2) ok = mbar_wait(bar(Lay::B_DQF + b), ((it >> 1) - 1) & 1, &s_wait, status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t sQ = sb + Lay::Q + s * Lay::QT, sDO = sb + Lay::DO + s * Lay::QT;
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it + 1 < nit) load_stats(i + 1, nl, nd);
       ok = named_barrier_and(kBarCompute, 128, ok);
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_abort, status));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_wait, status));
       float sv[64], dp[64];
       if (ok) {
         tc_fence_after();
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__any_sync(0xffffffffu, !(mf.x <= 65504.f && mf.y <= 65504.f)) && lane == 0)
           set_status(status, LH_ERR_RANGE);
         // P/dS buffer b is free once the products of sub-tile it-2 have completed
-        if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_abort,
+        if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_wait,
                                                             status));
       }
       if (ok) {
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // epilogue: dV and dK rows of this key tile (the products' accumulators are final after B_FIN)
     ok = named_barrier_and(kBarCompute, 128, ok);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FIN), 0, &s_abort, status));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FIN), 0, &s_wait, status));
     if (ok) {
       tc_fence_after();
 #pragma unroll
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = 0; it < nit; ++it) {
       const int b = it & 1, i = i0 + it;
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(Lay::B_MM + b), (it >> 1) & 1, &s_abort, status));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(Lay::B_MM + b), (it >> 1) & 1, &s_wait, status));
       float v[64];
       if (ok) {
         tc_fence_after();

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Lay = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
-  __shared__ int s_abort;
+  __shared__ WaitCtl s_wait;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkv = v1 ? nkv0 + 1 : nkv0;  // key tiles loaded (= those of query tile 1 when it exists)
 
   if (threadIdx.x == 0) {
-    s_abort = 0;
+    wait_ctl_init(&s_wait, status);
     mbar_init(bar(Lay::B_Q), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(Lay::B_KF + b), 1);
@@ -101,12 +101,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const int b = j & 1;
         const uint32_t ph = ((j >> 1) - 1) & 1;  // phase of the previous use of this stage
-        if (j >= 2) ok = mbar_wait(bar(Lay::B_KE + b), ph, &s_abort, status);
+        if (j >= 2) ok = mbar_wait(bar(Lay::B_KE + b), ph, &s_wait, status);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(Lay::B_KF + b), Lay::TILE);
         for (int db = 0; db < D / 64; ++db)
           tma_load_3d(sb + Lay::K + b * Lay::TILE + db * 16384, &tmK, bar(Lay::B_KF + b), db * 64, j * kTile, bh);
-        if (j >= 2) ok = mbar_wait(bar(Lay::B_VE + b), ph, &s_abort, status);
+        if (j >= 2) ok = mbar_wait(bar(Lay::B_VE + b), ph, &s_wait, status);
         if (!ok) {
           kv_issued = j;  // K_j in flight without its V
           mbar_wait_teardown(bar(Lay::B_KF + b), (j >> 1) & 1);
@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ts(tO, tP + kk * 8, sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
                   (j > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar(Lay::B_Q), 0, &s_abort, status);
-      if (ok) ok = mbar_wait(bar(Lay::B_KF), 0, &s_abort, status);
+      bool ok = mbar_wait(bar(Lay::B_Q), 0, &s_wait, status);
+      if (ok) ok = mbar_wait(bar(Lay::B_KF), 0, &s_wait, status);
       if (ok) {
         tc_fence_after();
         mma_s(0, 0);
@@ -160,23 +160,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const int b = j & 1;
         const int nx = j + 1;
-        ok = mbar_wait(bar(Lay::B_VF + b), (j >> 1) & 1, &s_abort, status);
+        ok = mbar_wait(bar(Lay::B_VF + b), (j >> 1) & 1, &s_wait, status);
         if (ok && j < nkv0) {
-          ok = mbar_wait(bar(Lay::B_PF + 0), j & 1, &s_abort, status);
+          ok = mbar_wait(bar(Lay::B_PF + 0), j & 1, &s_wait, status);
           if (ok) {
             tc_fence_after();
             mma_pv(0, j);
           }
         }
         if (ok && nx < nkv) {
-          ok = mbar_wait(bar(Lay::B_KF + (nx & 1)), (nx >> 1) & 1, &s_abort, status);
+          ok = mbar_wait(bar(Lay::B_KF + (nx & 1)), (nx >> 1) & 1, &s_wait, status);
           if (ok && nx < nkv0) {
             tc_fence_after();
             mma_s(0, nx);
           }
         }
         if (ok && v1) {
-          ok = mbar_wait(bar(Lay::B_PF + 1), j & 1, &s_abort, status);
+          ok = mbar_wait(bar(Lay::B_PF + 1), j & 1, &s_wait, status);
           if (ok) {
             tc_fence_after();
             mma_pv(1, j);
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv_q && ok; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + q), j & 1, &s_abort, status));  // warp-uniform
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + q), j & 1, &s_wait, status));  // warp-uniform
         if (!ok) break;
         tc_fence_after();
         float s[4][32];
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       }
       // epilogue: wait for the last product, normalise, store
-      if (ok) ok = mbar_wait(bar(Lay::B_OD + q), 0, &s_abort, status);
+      if (ok) ok = mbar_wait(bar(Lay::B_OD + q), 0, &s_wait, status);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "lh.h"
 
 namespace {
@@ -61,17 +63,25 @@ constexpr int kMaxDevices = 64;
 StepEvents g_events[kMaxDevices];
 
 int events_for_current_device(StepEvents** out) {
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LH_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
   StepEvents& e = g_events[dev];
   if (!e.ready) {
-    const unsigned fl = cudaEventDisableTiming;
-    if (cudaEventCreateWithFlags(&e.start, fl) != cudaSuccess) return LH_ERR_CUDA;
-    for (int s = 0; s < kSlots; ++s)
-      if (cudaEventCreateWithFlags(&e.h2d[s], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&e.comp[s], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&e.d2h[s], fl) != cudaSuccess)
+    // create all events or none: on a failure the ones already created are destroyed
+    cudaEvent_t* all[1 + 3 * kSlots] = {&e.start};
+    for (int s = 0; s < kSlots; ++s) {
+      all[1 + 3 * s] = &e.h2d[s];
+      all[2 + 3 * s] = &e.comp[s];
+      all[3 + 3 * s] = &e.d2h[s];
+    }
+    for (int i = 0; i < 1 + 3 * kSlots; ++i) {
+      if (cudaEventCreateWithFlags(all[i], cudaEventDisableTiming) != cudaSuccess) {
+        for (int j = 0; j < i; ++j) cudaEventDestroy(*all[j]);
         return LH_ERR_CUDA;
+      }
+    }
     e.ready = true;
   }
   *out = &e;

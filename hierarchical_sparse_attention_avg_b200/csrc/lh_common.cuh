@@ -26,16 +26,19 @@ struct LhDims {
   int BH;
   int S;
   int R;       // slot rows per head: sum_l N_l
-  int Rs;      // score rows per head: sum_{l<=L-2} N_l
+  int Rs;      // score rows per head: sum of N_l over the scored levels
   int Rp;      // pyramid rows per head: sum_{l>=1} N_l
-  int Ksel;    // selection-list rows per head: sum over partially selected levels of k
-  int nPartial;  // levels 0..nPartial-1 are partially selected (k < N_l); the rest are kept whole
+  int Ksel;    // selection-list rows per head: sum over partially selected levels of kl
+  int nPartial;  // levels 0..nPartial-1 are partially selected; the rest are kept whole
+  int expand;    // children-expansion variant (LH_EXPAND_CHILDREN): level l keeps the children of level l+1's picks
+  unsigned score_mask;  // bit l set: level l is scored (0..L-2, or 1..L-1 with expand)
   int Nl[LH_MAX_LEVELS];     // entries of level l
   int wl[LH_MAX_LEVELS];     // tokens per entry of level l
   int wlog[LH_MAX_LEVELS];   // log2(wl[l]) (windows are powers of two for every supported p)
   int off[LH_MAX_LEVELS];    // global pyramid id (= slot row) of entry (l, 0)
   int poff[LH_MAX_LEVELS];   // row of level l (>= 1) inside the per-head pyramid of lh_pool
   int kl[LH_MAX_LEVELS];     // selected entries of level l
+  int soff[LH_MAX_LEVELS];   // row of scored level l inside the per-head score array
   int seloff[LH_MAX_LEVELS]; // row of level l inside the per-head selection list (partial levels only)
   int* status;               // device status word of the current device (first error wins)
 };
@@ -51,8 +54,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// A wait gives up after this many nanoseconds and records LH_ERR_TIMEOUT.
+// Bound of the waits taken while tearing down after an abort (they wait for the block's own copies and products,
+// which always complete).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// The device status word is the first member of this per-device record; the kernels receive a pointer to it.  The
+// record also holds the bound on every ordinary device-side wait (lh_set_wait_limit_ns; 2 s by default).
+struct LhDeviceState {
+  int status;
+  int pad;
+  unsigned long long wait_limit_ns;
+};
+__device__ __forceinline__ uint64_t wait_limit_ns(const int* status) {
+  return reinterpret_cast<const volatile LhDeviceState*>(status)->wait_limit_ns;
+}
 
 // ------------------------------------------------------------------------------------------------------------
 // Number formats.
@@ -185,21 +200,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier.  Returns false (and records LH_ERR_TIMEOUT) when the wait exceeds
-// kWaitLimitNs, or immediately once `abort` (shared flag) is set by another thread of the block.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking test of the completion of phase `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Per-block wait control in shared memory: the abort flag (set by the first wait that gives up, so that every
+// other wait of the block returns at once) and the wait limit, read once from the device record at block start.
+struct WaitCtl {
+  int abort;
+  int pad;
+  unsigned long long limit_ns;
+};
+__device__ __forceinline__ void wait_ctl_init(WaitCtl* w, const int* status) {
+  w->abort = 0;
+  w->limit_ns = wait_limit_ns(status);
+}
+
+// Wait for phase `parity` of an mbarrier.  Returns false (and records LH_ERR_TIMEOUT) once the wait has lasted
+// longer than the block's wait limit, or immediately once the block's abort flag is set.  The elapsed time is checked
+// before each blocking try, so a limit of 1 ns makes every wait that finds its phase incomplete give up at once.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* w, int* status) {
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        set_status(status, LH_ERR_TIMEOUT);
-        *abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (w->abort) return false;
+    const uint64_t limit = w->limit_ns;
+    if (limit <= 1 || globaltimer_ns() - t0 > limit) {
+      set_status(status, LH_ERR_TIMEOUT);
+      w->abort = 1;
+      return false;
     }
+    if (mbar_try_wait(bar, parity)) return true;
   }
 }
 

@@ -90,7 +90,9 @@ __device__ __forceinline__ bool zero_or_normal(float x) {
 // coarsest entry): level 1 as above, levels >= 2 in fp64 registers, in the order the definition fixes.  The raw
 // rows stream through kPoolStages batches of TB rows per thread, copied with cp.async into shared-memory slots
 // private to the thread (so no block barrier is needed) while earlier batches are summed.
-template <int D, int P, int L, bool kScore>
+// kScore: 0 = no scores; 1 = score levels 0..L-2; 2 = score levels 1..L-1 (children-expansion variant).  Scored
+// level l is written at row dm.soff[l] of the head's score array.
+template <int D, int P, int L, int kScore>
 __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, LhDims dm) {
   constexpr int G = D / 8;
   constexpr int GPB = kPoolThreads / G;
@@ -144,12 +146,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
       for (int c = 0; c < P; ++c) {
         float xf[8];
         unpack8(raw_s[(g1 * P + c) * kPoolThreads], xf);
-        if (kScore) {  // level 0 is scored whenever L >= 2
+        if (kScore == 1) {  // level 0 is scored whenever L >= 2 (not in the children-expansion variant)
           double x[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) x[i] = f64_of(xf[i]);
           float s = row_score<G>(x);
-          if (active && lane == 0) scores[dm.off[0] + (int64_t)blk * W + t0 + g1 * P + c] = s;
+          if (active && lane == 0) scores[dm.soff[0] + (int64_t)blk * W + t0 + g1 * P + c] = s;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
       for (int i = 0; i < 8; ++i) exact &= same_sum(up[i], dn[i]);
       const int j1 = blk * (W / P) + t0 / P + g1;  // global level-1 index
       const bool write1 = (job.write_mask >> 1) & 1u;
-      const bool score1 = kScore && 1 <= L - 2;
+      const bool score1 = (kScore == 1 && 1 <= L - 2) || kScore == 2;
       // the fp64 level-1 sum: needed above level 1, and for the rounding when the fp32 one is not exact
       if (!exact) {
 #pragma unroll
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
 #pragma unroll
           for (int i = 0; i < 8; ++i) v[i] = f64_of(vf[i]);
           const float sc = row_score<G>(v);
-          if (active && lane == 0) scores[dm.off[1] + j1] = sc;
+          if (active && lane == 0) scores[dm.soff[1] + j1] = sc;
         }
       }
       // levels >= 2: walk up while parents complete
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
         jloc /= P;
         const int64_t j = (int64_t)blk * (W / ipow(P, lev)) + jloc;  // global index at level lev
         const bool write = (job.write_mask >> lev) & 1u;
-        const bool score = kScore && lev <= L - 2;
+        const bool score = (kScore == 1 && lev <= L - 2) || kScore == 2;
         if (write || score) {
           double val[8];
           const uint4 packed = round_pooled(acc[lev], 1.0 / (double)ipow(P, lev), val);
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
             st16(pyr + ((int64_t)bh * job.pyr_rows + job.row_off[lev] + j) * D + lane * 8, packed);
           if (score) {
             float s = row_score<G>(val);
-            if (active && lane == 0) scores[dm.off[lev] + j] = s;
+            if (active && lane == 0) scores[dm.soff[lev] + j] = s;
           }
         }
       }
@@ -506,12 +508,12 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherJobs jo
 
 // Jobs with scores and jobs without run as two launches of the two specialisations (the one without carries no
 // scoring code and fewer registers).
-template <int D, int P, int L, bool kScore>
+template <int D, int P, int L, int kScore>
 int launch_pool_kind(const PoolJobs& all, int njobs, const LhDims& dm, cudaStream_t st) {
   PoolJobs jobs;
   int n = 0;
   for (int i = 0; i < njobs; ++i)
-    if ((all.job[i].scores != nullptr) == kScore) jobs.job[n++] = all.job[i];
+    if ((all.job[i].scores != nullptr) == (kScore != 0)) jobs.job[n++] = all.job[i];
   if (n == 0) return LH_OK;
   constexpr int G = D / 8;
   constexpr int W = ipow(P, L - 1);
@@ -528,8 +530,9 @@ int launch_pool_kind(const PoolJobs& all, int njobs, const LhDims& dm, cudaStrea
 
 template <int D, int P, int L>
 int launch_pool_t(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
-  const int rc = launch_pool_kind<D, P, L, false>(jobs, njobs, dm, st);
-  return rc != LH_OK ? rc : launch_pool_kind<D, P, L, true>(jobs, njobs, dm, st);
+  const int rc = launch_pool_kind<D, P, L, 0>(jobs, njobs, dm, st);
+  if (rc != LH_OK) return rc;
+  return dm.expand ? launch_pool_kind<D, P, L, 2>(jobs, njobs, dm, st) : launch_pool_kind<D, P, L, 1>(jobs, njobs, dm, st);
 }
 
 template <int D, int P>

@@ -60,12 +60,16 @@ __device__ __forceinline__ void head_max_atomic(float m, int bh, bool active, in
   }
 }
 
-// Power-of-two scale bringing the largest magnitude `amax` into [2^9, 2^10); 1 for an all-zero head.
+// Power-of-two scale bringing the largest magnitude `amax` into [2^9, 2^10); 1 for an all-zero or non-finite head.
+// The exponent is read from the bits and the scale is capped at 2^126, so that both the scale and its inverse stay
+// finite normal fp32 numbers: a head whose largest magnitude is below 2^-116 (subnormal values included) is scaled
+// by 2^126 and keeps its values below 2^10.
 __device__ __forceinline__ float head_scale(float amax) {
   if (!(amax > 0.f) || !isfinite(amax)) return 1.f;
-  int e;
-  frexpf(amax, &e);  // amax = m 2^e, m in [0.5, 1)
-  return ldexpf(1.f, 10 - e);
+  const int biased = (int)((__float_as_uint(amax) >> 23) & 0xFFu);  // 0 for a subnormal amax
+  const int e = (biased == 0 ? -126 : biased - 127) + 1;               // amax < 2^e
+  const int s = 10 - e < 126 ? 10 - e : 126;
+  return __uint_as_float((uint32_t)(s + 127) << 23);
 }
 
 // Window sums for the scatter-back (offset, one tensor) and the unpool backward (three tensors).

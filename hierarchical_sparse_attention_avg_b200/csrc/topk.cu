@@ -3,11 +3,14 @@
 // Selection follows [W] 核心方法 §2 ("Chunked Bitonic Top-K" kernel) and [C] "Four-Stage Pipeline Wraps Standard
 // FlashAttention" (per-level stratified top-K, coarsest level always kept whole): every level l <= L-2 with fewer
 // picks than entries is cut into C equal contiguous chunks, and each chunk keeps its k/C entries of largest
-// score, ties to the lower index.
+// score, ties to the lower index.  In the children-expansion variant (the reading that reproduces the size example
+// of [E] "Какво точно промени Nous Research в attention пътя?") the chunks and scores are those of level l+1, and
+// level l keeps the p children of every pick.
 //
-// Keys: a score is non-negative, so its fp32 bit pattern orders like the value; key = (score bits << 32) |
-// (0xFFFFFFFF - index) is unique, and a larger key means a higher score or, on equal scores, a lower index.
-// Sentinel key 0 is below every real key.
+// Keys: the score's fp32 bit pattern is mapped to an unsigned integer that orders like the value (negative numbers:
+// all bits flipped; others: sign bit set; -0 is first made +0, so that the two zeros tie); key = (ordered score
+// << 32) | (0xFFFFFFFF - index) is unique, and a larger key means a higher score or, on equal scores, a lower
+// index.  Sentinel key 0 is below every real key (the index part of a real key is never 0).
 //
 // One CTA (8 warps) per (head, level, chunk).  Each warp keeps a running top-M (M = picks rounded up to a power
 // of two) of its share of the chunk in registers, M/32 keys per lane, sorted descending.  Keys of the warp's
@@ -25,7 +28,10 @@ namespace lh {
 namespace {
 
 __device__ __forceinline__ uint64_t make_key(float score, uint32_t index) {
-  return ((uint64_t)__float_as_uint(score) << 32) | (uint64_t)(0xFFFFFFFFu - index);
+  uint32_t u = __float_as_uint(score);
+  if (u == 0x80000000u) u = 0u;  // -0 ties with +0
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - index);
 }
 __device__ __forceinline__ uint32_t key_index(uint64_t key) { return 0xFFFFFFFFu - (uint32_t)key; }
 
@@ -101,14 +107,18 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   __shared__ uint64_t s_top[8][M];
   __shared__ uint32_t s_idx[M];
 
+  // lev: the level whose selection list this block writes; rlev: the level whose entries it ranks (lev itself, or
+  // its parent level in the children-expansion variant, where each pick brings its p children at level lev)
   const int c = blockIdx.x, lev = blockIdx.y, bh = blockIdx.z;
-  const int nc = dm.Nl[lev] / dm.C;
-  const int m = dm.kl[lev] / dm.C;
+  const int rlev = lev + dm.expand;
+  const int nc = dm.Nl[rlev] / dm.C;
+  const int m = dm.k / dm.C;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const float* sc = scores + (int64_t)bh * dm.Rs + dm.off[lev] + (int64_t)c * nc;
-  int32_t* sl = slot + (int64_t)bh * dm.R + dm.off[lev] + (int64_t)c * nc;
+  const float* sc = scores + (int64_t)bh * dm.Rs + dm.soff[rlev] + (int64_t)c * nc;
+  const int nslot = dm.Nl[lev] / dm.C;  // entries of level lev in this chunk
+  int32_t* sl = slot + (int64_t)bh * dm.R + dm.off[lev] + (int64_t)c * nslot;
 
-  for (int i = threadIdx.x; i < nc; i += 256) sl[i] = -1;  // positions of the picks are written later
+  for (int i = threadIdx.x; i < nslot; i += 256) sl[i] = -1;  // positions of the picks are written later
 
   uint64_t top[R];
 #pragma unroll
@@ -172,12 +182,15 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
     for (int r = 0; r < R; ++r) s_idx[lane * R + r] = key_index(top[r]);
   }
   __syncthreads();
-  // the first m keys are the picks; emit their indices in ascending order (rank = number of smaller indices)
+  // the first m keys are the picks; emit their indices in ascending order (rank = number of smaller indices), or,
+  // in the children-expansion variant, the p children of each pick (consecutive, so the list stays ascending)
+  const int fan = dm.expand ? dm.p : 1;
   for (int i = threadIdx.x; i < m; i += 256) {
     const uint32_t me = s_idx[i];
     int rank = 0;
     for (int q = 0; q < m; ++q) rank += s_idx[q] < me;
-    sel[(int64_t)bh * dm.Ksel + dm.seloff[lev] + c * m + rank] = (int32_t)me;
+    int32_t* dst = sel + (int64_t)bh * dm.Ksel + dm.seloff[lev] + ((int64_t)c * m + rank) * fan;
+    for (int e = 0; e < fan; ++e) dst[e] = (int32_t)me * fan + e;
   }
 }
 

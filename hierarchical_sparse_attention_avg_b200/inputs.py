@@ -40,15 +40,23 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int = 0, device="cpu", wit
     return q, k, v, dout
 
 
-def make_scores(B: int, H: int, rows: int, seed: int = 0, device="cpu", ties: bool = False) -> torch.Tensor:
-    """Non-negative fp32 scores ``[B, H, rows]`` for feeding the top-K step directly.
+def make_scores(B: int, H: int, rows: int, seed: int = 0, device="cpu", ties: bool = False,
+                signed: bool = False) -> torch.Tensor:
+    """fp32 scores ``[B, H, rows]`` for feeding the top-K step directly: non-negative by default.
 
     With ``ties=True`` the values are drawn from a small set so that many scores are equal, which exercises the
-    lower-index tie rule."""
+    lower-index tie rule.  With ``signed=True`` they are N(0, 1) values of both signs, about one in eight replaced
+    by a zero of random sign (so that -0 meets +0) and one in eight by a value repeated across the row."""
     g = _generator(seed, device)
     if ties:
         return torch.randint(0, 4, (B, H, rows), generator=g, device=device).to(torch.float32)
     z = torch.randn((B, H, rows), generator=g, device=device, dtype=torch.float32)
+    if signed:
+        u = torch.rand((B, H, rows), generator=g, device=device)
+        sign = torch.randint(0, 2, (B, H, rows), generator=g, device=device).to(torch.float32) * 2 - 1
+        z = torch.where(u < 0.125, sign * 0.0, z)
+        z = torch.where((u >= 0.125) & (u < 0.25), torch.full_like(z, -0.75), z)
+        return z
     return z * z
 
 

@@ -23,6 +23,8 @@ LH_ERR_TIMEOUT = 4
 LH_ERR_WORKSPACE = 5
 LH_ERR_RANGE = 6
 
+LH_EXPAND_CHILDREN = 1
+
 
 class LhParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "L", "p", "k", "C", "flags")]
@@ -66,6 +68,7 @@ _SIGS = {
     "lh_scatter_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp]),
     "lh_attend_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "lh_get_status": (ctypes.c_int, [_vp]),
+    "lh_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "lh_score_topk_static": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
     "lh_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "lh_profile_read": (ctypes.c_int, [ctypes.POINTER(LhKernelTime), ctypes.c_int]),
@@ -107,9 +110,11 @@ class Params:
     p: int
     k: int
     C: int
+    expand: bool = False  # LH_EXPAND_CHILDREN
 
     def c(self) -> LhParams:
-        return LhParams(self.B, self.H, self.N, self.d, self.L, self.p, self.k, self.C, 0)
+        return LhParams(self.B, self.H, self.N, self.d, self.L, self.p, self.k, self.C,
+                        LH_EXPAND_CHILDREN if self.expand else 0)
 
 
 def error_string(status: int) -> str:
@@ -409,6 +414,13 @@ def lh_attend_bwd(P: Params, qg, kg, vg, og, lse, dog, ws=None):
 def lh_get_status(device=None) -> int:
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     return _lib.lh_get_status(_stream(dev))
+
+
+def lh_set_wait_limit_ns(ns: int, device=None) -> None:
+    """Bound on every device-side wait of later launches on ``device`` (0 restores the default of 2 s)."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(_lib.lh_set_wait_limit_ns(int(ns)), "lh_set_wait_limit_ns")
 
 
 def lh_profile_enable(on: bool = True) -> None:

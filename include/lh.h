@@ -22,7 +22,8 @@
  *   - Sizes: B batch, H heads, N tokens, d head dim, L levels, p pool factor, k picks per level, C chunks per
  *     level.  w_l = p^l, N_l = N / w_l.  S = sum_{l<=L-2} min(k, N_l) + N_{L-1}.
  *   - Global pyramid id of entry (l, j): off_l + j with off_l = sum_{l'<l} N_l' (level 0 = raw tokens first).
- *   - The library never allocates device memory, never synchronises (except lh_get_status) and never throws.
+ *   - The library never allocates device memory, never synchronises (except lh_get_status and
+ *     lh_set_wait_limit_ns) and never throws.
  *     Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default stream).
  *   - Scratch memory is the caller's `ws` of at least lh_workspace_bytes(P) bytes.
  *   - Return value: LH_OK, or an error code.  Argument errors are detected on the host before any launch.
@@ -51,7 +52,17 @@ extern "C" {
 
 #define LH_MAX_LEVELS 8
 
-/* Layer sizes.  flags is reserved and must be 0. */
+/* lh_params.flags: LH_EXPAND_CHILDREN selects the children-expansion reading of the selection, the one under which
+ * the size example of [E] "Какво точно промени Nous Research в attention пътя?" (N = 1,000,000, L = 4, p = 4,
+ * k = 4,096 -> a gathered sequence of about 65,000 tokens) comes out: the keys of levels 1..L-1 are scored, the
+ * chunked top-K ranks level l+1 (C chunks, k/C picks each, ties to the lower index), and level l <= L-2 keeps the
+ * p children p*J .. p*J + p-1 of every pick J; the coarsest level is still kept whole.  Then
+ * S = sum_{l=1}^{L-1} p*min(k, N_l) + N_{L-1} (64,777 at that example; 65,536 at N = 2^20).  Validity: C | N_l and
+ * C | k for every ranked level l with k < N_l.  Everything after the selection (order, gather, attention,
+ * scatter, backward) is unchanged.  flags = 0 is the per-level reading of the conventions above. */
+#define LH_EXPAND_CHILDREN 1
+
+/* Layer sizes.  flags: 0 or LH_EXPAND_CHILDREN (any other bit is LH_ERR_INVALID_ARG). */
 typedef struct lh_params {
   int32_t B, H, N, d, L, p, k, C;
   int32_t flags;
@@ -90,7 +101,8 @@ int64_t lh_level_offset(const lh_params* P, int level);
  * sum_{1<=l'<l} N_l'); -1 if invalid. */
 int64_t lh_pyramid_rows(const lh_params* P);
 
-/* Rows per head of the score array: sum_{l=0}^{L-2} N_l (level l starts at row off_l); -1 if invalid. */
+/* Rows per head of the score array: sum_{l=0}^{L-2} N_l (level l starts at row off_l); with LH_EXPAND_CHILDREN
+ * sum_{l=1}^{L-1} N_l (level l starts at row off_l - N_0); -1 if invalid. */
 int64_t lh_score_rows(const lh_params* P);
 
 /* Rows per head of the slot map: sum_{l=0}^{L-1} N_l; -1 if invalid. */
@@ -117,8 +129,10 @@ int lh_pool(const lh_params* P, const void* x, void* pyr, void* stream);
  * FlashAttention").
  * k: bf16 [B,H,N,d] raw keys.  Scores: squared l2 norm of the pooled key (raw key at level 0), fp64 sum of
  * squares (eight left to right per group of eight features, then a pairwise tree over the groups), rounded
- * to fp32, for levels 0..L-2.
- * scores_in: optional fp32 [B,H,lh_score_rows]; when non-NULL it replaces the computed scores.
+ * to fp32, for levels 0..L-2 (levels 1..L-1 with LH_EXPAND_CHILDREN).
+ * scores_in: optional fp32 [B,H,lh_score_rows]; when non-NULL it replaces the computed scores.  Any finite values
+ * are ordered correctly (negative ones included; -0 and +0 are equal and tie); NaN scores give an unspecified but
+ * deterministic selection.
  * scores_out: optional fp32 [B,H,lh_score_rows]; when non-NULL (and scores_in is NULL) receives the scores.
  * Selection: C equal chunks per level, each keeping its min(k,N_l)/C entries of largest score (ties: lower
  * index); coarsest level whole.  Order: ascending end token (j+1)*p^l - 1, equal ends coarser level first.
@@ -159,7 +173,9 @@ int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, 
 
 /* Whole backward ([E] "Как four-stage pipeline…": gradients reach Q, K, V only through the gathered values;
  * [W] 深度洞察).  dout: bf16 [B,H,N,d]; ctx from lh_forward; dq,dk,dv: bf16 [B,H,N,d] (out).
- * dX[t] = sum_l [(l, floor(t/p^l)) selected] dX_g[slot] / p^l. */
+ * dX[t] = sum_l [(l, floor(t/p^l)) selected] dX_g[slot] / p^l.
+ * Determinism: dk and dv are bitwise reproducible from run to run; dq is accumulated with fp32 reduce-adds whose
+ * order is not fixed, so it may differ in its last bits between runs (always within the stated tolerance). */
 int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq, void* dk, void* dv, void* ws,
                 size_t ws_bytes, void* stream);
 
@@ -194,8 +210,9 @@ int lh_profile_read(lh_kernel_time_t* out, int max_entries);
 
 /* ---- selection without caller scratch ---------------------------------------------------------------- */
 
-/* Size of the library's fixed device scratch array used by lh_score_topk_static (per device, held from the
- * first use of the library on that device until the process exits). */
+/* Size of the library's fixed device scratch array used by lh_score_topk_static.  No call allocates it: it is part
+ * of the library's device module, so every device on which the library's kernels are loaded (the first use of any
+ * entry point there) reserves these bytes until the process exits, whether or not lh_score_topk_static is called. */
 #define LH_STATIC_SCRATCH_BYTES (16u << 20)
 
 /* The pages have no counterpart to this entry point; it exists for callers that cannot allocate device memory
@@ -238,8 +255,8 @@ size_t lh_step_host_bytes(const lh_params* P, int heads_per_chunk);
  * makes o, dq, dk, dv valid on the host.  Errors: LH_ERR_INVALID_ARG (sizes, heads_per_chunk, NULL or misaligned
  * pointers), LH_ERR_WORKSPACE (dev_bytes too small), LH_ERR_CUDA (a copy, event or launch failed), or the error
  * of lh_forward / lh_backward; a failure mid-way leaves the earlier chunks enqueued.  The pipeline's events are
- * created on the first call on each device and reused, so concurrent calls on one device from several host
- * threads must be serialised by the caller. */
+ * created once per device (the first call, under a lock) and reused by every call, so calls on one device whose
+ * work can overlap (several host threads or streams) must be serialised by the caller. */
 int lh_step_host(const lh_params* P, const void* q, const void* k, const void* v, const void* dout, void* o, void* dq,
                  void* dk, void* dv, int heads_per_chunk, void* dev, size_t dev_bytes, void* stream, void* h2d_stream,
                  void* d2h_stream);
@@ -249,6 +266,14 @@ int lh_step_host(const lh_params* P, const void* q, const void* k, const void* v
 /* Synchronises `stream`, returns the first device-side error recorded since the last call (LH_OK if none)
  * on the current device, and clears it. */
 int lh_get_status(void* stream);
+
+/* Bound, in nanoseconds, on every device-side wait of the kernels launched on the current device from now on
+ * (0 restores the default of 2 s).  A wait that exceeds it records LH_ERR_TIMEOUT (read with lh_get_status); the
+ * block then stops, after waiting for the copies and tensor-core products it has issued, and frees its tensor
+ * memory, so the context stays usable and the next call computes normally.  It exists to test that path: a short
+ * limit makes ordinary waits give up.  Synchronises the device (call it while no other work of the library is in
+ * flight); LH_OK or LH_ERR_CUDA. */
+int lh_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

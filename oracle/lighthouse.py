@@ -49,6 +49,7 @@ class Params:
     p: int
     k: int
     C: int
+    expand: bool = False
 
     def window(self, lev: int) -> int:
         """Tokens covered by one entry of level ``lev``: ``p**lev``."""
@@ -62,14 +63,34 @@ class Params:
         """Entries kept at level ``lev``: ``min(k, N_lev)`` below the coarsest level, all of the coarsest.
 
         Reading: "top-K per level" with the coarsest level "always retained in full" ([C] "Four-Stage
-        Pipeline…")."""
+        Pipeline…").  With ``expand`` (the children-expansion variant): ``p * min(k, N_{lev+1})`` below the
+        coarsest level, the children of the entries picked one level up."""
         if lev == self.L - 1:
             return self.level_size(lev)
+        if self.expand:
+            return self.p * self.parent_picks(lev + 1)
         return min(self.k, self.level_size(lev))
 
+    def parent_picks(self, lev: int) -> int:
+        """Children-expansion variant: entries of level ``lev`` (1 .. L-1) picked by score, ``min(k, N_lev)``."""
+        return min(self.k, self.level_size(lev))
+
+    def scored_levels(self) -> list[int]:
+        """Levels whose pooled keys are scored: ``0 .. L-2``, or ``1 .. L-1`` in the children-expansion variant."""
+        return list(range(1, self.L)) if self.expand else list(range(self.L - 1))
+
     def gathered_length(self) -> int:
-        """``S = sum_{lev <= L-2} min(k, N_lev) + N_{L-1}`` (reading R-S)."""
+        """``S = sum_{lev <= L-2} min(k, N_lev) + N_{L-1}`` (reading R-S), or, in the children-expansion variant,
+        ``S = sum_{lev=1}^{L-1} p * min(k, N_lev) + N_{L-1}``."""
         return sum(self.picks(lev) for lev in range(self.L))
+
+    def score_rows(self) -> int:
+        """Rows of one head's score array: the scored levels concatenated, finest first."""
+        return sum(self.level_size(x) for x in self.scored_levels())
+
+    def score_offset(self, lev: int) -> int:
+        """Row of scored level ``lev``'s first entry in one head's score array."""
+        return sum(self.level_size(x) for x in self.scored_levels() if x < lev)
 
     def level_offset(self, lev: int) -> int:
         """Global pyramid id of entry ``(lev, 0)``: number of entries of all finer levels."""
@@ -83,11 +104,14 @@ class Params:
         if self.d % 8 or (self.d // 8) & (self.d // 8 - 1):
             raise ValueError("d must be 8 times a power of two (score summation order)")
         for lev in range(self.L - 1):
-            n, kk = self.level_size(lev), self.picks(lev)
+            if self.expand:
+                n, kk = self.level_size(lev + 1), self.parent_picks(lev + 1)
+            else:
+                n, kk = self.level_size(lev), self.picks(lev)
             if kk == n:
                 continue
             if n % self.C or kk % self.C:
-                raise ValueError(f"C must divide N_{lev} and k_{lev}")
+                raise ValueError(f"C must divide the entries and the picks of every partially picked level")
 
 
 # --------------------------------------------------------------------------------------------------------------
@@ -172,13 +196,13 @@ def pyramid(x: np.ndarray, P: Params, round_pool: bool = True) -> list[np.ndarra
 # --------------------------------------------------------------------------------------------------------------
 
 def norm_scores(kpyr: list[np.ndarray], P: Params) -> list[np.ndarray]:
-    """Squared l2 norm of every pooled key of levels ``0 .. L-2``, as float32.
+    """Squared l2 norm of every pooled key of the scored levels (``P.scored_levels()``), as float32.
 
     [W] 核心方法 §2 and [E] "Как four-stage pipeline…" score entries with a parameter-free per-head l2 norm.
     Reading P2: the norm of the pooled key, squared (same order as the norm).  Summation order: eight squares
     left to right per group of eight features, then a pairwise tree over the groups; one rounding to fp32."""
     out = []
-    for lev in range(P.L - 1):
+    for lev in P.scored_levels():
         sq = kpyr[lev] * kpyr[lev]                      # exact in float64 (16-bit significands)
         groups = sq.reshape(sq.shape[0], P.d // 8, 8)
         part = groups[:, :, 0].copy()
@@ -194,27 +218,52 @@ def norm_scores(kpyr: list[np.ndarray], P: Params) -> list[np.ndarray]:
 # Step 3: stratified (chunked) top-K per level, coarsest level kept whole
 # --------------------------------------------------------------------------------------------------------------
 
+def chunked_top(s: np.ndarray, picks: int, P: Params) -> np.ndarray:
+    """Indices, ascending, of the ``picks`` entries of largest score of one level split into ``C`` equal
+    contiguous chunks, ``picks / C`` from each chunk, ties to the lower index (found by sorting each chunk)."""
+    s = np.asarray(s, dtype=np.float64)
+    n = len(s)
+    n_c, m = n // P.C, picks // P.C
+    chosen = []
+    for c in range(P.C):
+        j = np.arange(c * n_c, (c + 1) * n_c, dtype=np.int64)
+        order = np.lexsort((j, -s[j]))             # primary: score descending; secondary: index ascending
+        chosen.append(np.sort(j[order[:m]]))
+    return np.concatenate(chosen)
+
+
 def select(scores: list[np.ndarray], P: Params) -> list[np.ndarray]:
-    """Selected entry indices of every level, ascending.
+    """Selected entry indices of every level, ascending.  ``scores[i]`` belongs to level ``P.scored_levels()[i]``.
 
     Levels ``0 .. L-2``: ``C`` equal contiguous chunks, each keeping its ``k_lev / C`` entries with the largest
     score, ties to the lower index, found by sorting each chunk ([W] 核心方法 §2 "Chunked Bitonic Top-K";
     [C] "Four-Stage Pipeline…": stratified rather than global top-K).  When ``k >= N_lev`` the whole level is
-    kept.  The coarsest level is always kept whole ([C] "Four-Stage Pipeline…")."""
+    kept.  The coarsest level is always kept whole ([C] "Four-Stage Pipeline…").
+
+    Children-expansion variant (``P.expand``; the reading under which the size example of [E] "Какво точно
+    промени Nous Research в attention пътя?" comes out): the chunked top-K runs on the scored levels
+    ``1 .. L-1``, and level ``lev <= L-2`` keeps the ``p`` children ``p*J .. p*J + p-1`` of every entry ``J``
+    picked at level ``lev + 1``; the coarsest level is still kept whole."""
+    if P.expand:
+        sel = []
+        for lev in range(P.L - 1):
+            parent = lev + 1
+            n_par = P.level_size(parent)
+            if P.parent_picks(parent) == n_par:
+                sel.append(np.arange(P.level_size(lev), dtype=np.int64))
+                continue
+            J = chunked_top(scores[parent - 1], P.parent_picks(parent), P)
+            kids = (J[:, None] * P.p + np.arange(P.p, dtype=np.int64)[None, :]).reshape(-1)
+            sel.append(kids)
+        sel.append(np.arange(P.level_size(P.L - 1), dtype=np.int64))
+        return sel
     sel = []
     for lev in range(P.L):
         n = P.level_size(lev)
         if lev == P.L - 1 or P.picks(lev) == n:
             sel.append(np.arange(n, dtype=np.int64))
             continue
-        s = np.asarray(scores[lev], dtype=np.float64)
-        n_c, m = n // P.C, P.picks(lev) // P.C
-        chosen = []
-        for c in range(P.C):
-            j = np.arange(c * n_c, (c + 1) * n_c, dtype=np.int64)
-            order = np.lexsort((j, -s[j]))             # primary: score descending; secondary: index ascending
-            chosen.append(np.sort(j[order[:m]]))
-        sel.append(np.concatenate(chosen))
+        sel.append(chunked_top(scores[lev], P.picks(lev), P))
     return sel
 
 

@@ -53,6 +53,10 @@ CONFIGS = [
     (1, 8, 1048576, 128, 4, 4, 4096, 32),
     (2, 3, 1024, 128, 1, 4, 100, 1),
     (1, 1, 512, 64, 5, 2, 8, 2),
+    # children-expansion variant: the pages' size example at N = 2^20, the 4K case, a whole-level case
+    (1, 8, 1048576, 128, 4, 4, 4096, 32, True),
+    (1, 2, 4096, 64, 3, 4, 64, 4, True),
+    (1, 1, 1024, 64, 3, 4, 64, 4, True),
 ]
 
 
@@ -66,7 +70,7 @@ def test_sizes_match_oracle(lh, cfg):
         assert lh.lh_level_offset(P, lev) == Q.level_offset(lev)
     assert lh.lh_level_size(P, Q.L) == -1
     assert lh.lh_pyramid_rows(P) == sum(Q.level_size(lev) for lev in range(1, Q.L))
-    assert lh.lh_score_rows(P) == sum(Q.level_size(lev) for lev in range(Q.L - 1))
+    assert lh.lh_score_rows(P) == Q.score_rows()
     assert lh.lh_slot_rows(P) == sum(Q.level_size(lev) for lev in range(Q.L))
     lay = lh.lh_ctx_layout(P)
     S, rows = Q.gathered_length(), Q.B * Q.H
@@ -91,6 +95,17 @@ def test_sizes_match_oracle(lh, cfg):
 ])
 def test_validation_codes(lh, cfg, code):
     assert lh.lh_validate(lh.Params(*cfg)) == code
+
+
+def test_expand_variant_sizes_and_validation(lh):
+    P = lh.Params(1, 8, 1048576, 128, 4, 4, 4096, 32, True)
+    assert lh.lh_S(P) == 65536                                   # 16,384 coarsest + 3 levels x 4 x 4,096
+    assert lh.lh_score_rows(P) == 262144 + 65536 + 16384          # levels 1..3 scored
+    assert lh.lh_validate(lh.Params(1, 1, 4096, 64, 3, 4, 64, 3, True)) == lh.LH_ERR_INVALID_ARG  # 3 does not divide
+    import ctypes as C
+    bad = lh.Params(1, 1, 4096, 64, 3, 4, 64, 4).c()
+    bad.flags = 2                                                # an unknown flag bit
+    assert lh.library().lh_validate(C.byref(bad)) == lh.LH_ERR_INVALID_ARG
 
 
 def test_k_at_least_level_size_needs_no_divisibility(lh):

@@ -27,6 +27,10 @@ CASES = {
     "p8-L3-B2": (2, 1, 4096, 128, 3, 8, 64, 4),
     # the pages' recipe parameters L=3, p=4, k=1536 ([C] "The Core Innovation"), C=16: 96 picks per chunk, S = 4096
     "recipe-L3-k1536": (1, 1, 16384, 64, 3, 4, 1536, 16),
+    # children-expansion variant (LH_EXPAND_CHILDREN): level l keeps the p children of level l+1's picks
+    "expand-L3-d64": (1, 2, 4096, 64, 3, 4, 64, 4, True),      # S = 256 + 256 + 256
+    "expand-L4-d128": (1, 2, 16384, 128, 4, 4, 128, 8, True),  # S = 3 x 512 + 256 = 1792
+    "expand-p2-L4-whole-top": (1, 1, 2048, 64, 4, 2, 256, 2, True),  # level 1 ranked, levels 2.. whole
 }
 
 
@@ -89,16 +93,16 @@ def test_topk_fed_oracle_scores_bit_exact(case):
     if Q.L == 1:
         pytest.skip("single level: no scores")
     dev = case["q"].device
-    for ties in (False, True):
-        sc = make_scores(Q.B, Q.H, lh.lh_score_rows(P), seed=3, ties=ties)
+    for kind in ("plain", "ties", "signed"):  # signed: negative scores and zeros of both signs (-0 ties with +0)
+        sc = make_scores(Q.B, Q.H, lh.lh_score_rows(P), seed=3, ties=kind == "ties", signed=kind == "signed")
         idx_g, slot = lh.lh_score_topk(P, case["k"], scores_in=sc.to(dev))
         for (b, h) in case["heads"]:
-            per = [sc[b, h, Q.level_offset(lev): Q.level_offset(lev) + Q.level_size(lev)].numpy()
-                   for lev in range(Q.L - 1)]
+            per = [sc[b, h, Q.score_offset(lev): Q.score_offset(lev) + Q.level_size(lev)].numpy()
+                   for lev in Q.scored_levels()]
             sel = O.select(per, Q)
             lev_g, j_g, slots = O.gathered_order(sel, Q)
-            assert np.array_equal(idx_g[b, h].cpu().numpy(), O.global_ids(lev_g, j_g, Q)), (ties, b, h)
-            assert np.array_equal(slot[b, h].cpu().numpy(), O.slot_map(slots)), (ties, b, h)
+            assert np.array_equal(idx_g[b, h].cpu().numpy(), O.global_ids(lev_g, j_g, Q)), (kind, b, h)
+            assert np.array_equal(slot[b, h].cpu().numpy(), O.slot_map(slots)), (kind, b, h)
 
 
 def _fp16(a):

@@ -132,3 +132,44 @@ def test_pin_catches_planted_mistake(monkeypatch, name, bad, pin):
     monkeypatch.setattr(O, name, bad)
     with pytest.raises(AssertionError):
         pin()
+
+
+# ---- children-expansion variant ------------------------------------------------------------------------------
+
+def _expand_select_children_shifted(scores, P):
+    sel = _REAL_SELECT(scores, P)
+    return [np.minimum(s + 1, P.level_size(lev) - 1) if lev < P.L - 1 else s for lev, s in enumerate(sel)]
+
+
+def _expand_select_lowest_parents(scores, P):
+    """Ranks the parents by ascending score (a dropped minus sign in the sort key)."""
+    out = []
+    for lev in range(P.L - 1):
+        n_par = P.level_size(lev + 1)
+        if P.parent_picks(lev + 1) == n_par:
+            out.append(np.arange(P.level_size(lev)))
+            continue
+        J = O.chunked_top(-np.asarray(scores[lev], dtype=np.float64), P.parent_picks(lev + 1), P)
+        out.append((J[:, None] * P.p + np.arange(P.p)[None, :]).reshape(-1))
+    out.append(np.arange(P.level_size(P.L - 1)))
+    return out
+
+
+_REAL_SELECT = O.select
+
+
+@pytest.mark.parametrize("mutant", [_expand_select_children_shifted, _expand_select_lowest_parents])
+def test_expand_pins_catch_selection_mutants(monkeypatch, mutant):
+    def patched(scores, P):
+        return mutant(scores, P) if P.expand else _REAL_SELECT(scores, P)
+
+    monkeypatch.setattr(O, "select", patched)
+    failed = 0
+    for fn, args in ((pins.test_expand_selection_is_the_children_of_the_per_level_selection_one_level_up,
+                      (3, 4, 8, 2)),
+                     (pins.test_expand_selection_comes_in_sibling_groups_with_equal_counts_per_chunk, ())):
+        try:
+            fn(*args)
+        except AssertionError:
+            failed += 1
+    assert failed >= 1

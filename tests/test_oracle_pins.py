@@ -212,6 +212,78 @@ def test_pages_size_example_is_not_reproduced_by_the_per_level_reading():
 
 
 # ----------------------------------------------------------------------------------------------------------------
+# The children-expansion variant ([E] "Какво точно промени Nous Research в attention пътя?": the size example)
+# ----------------------------------------------------------------------------------------------------------------
+
+def test_expand_gathered_length_reproduces_the_pages_size_example():
+    g = json.load(open(os.path.join(HERE, "golden", "pages_size_example.json")))
+    N, L, p, k = g["N"], g["L"], g["p"], g["k"]
+    P = O.Params(1, 1, N, 8, L, p, k, 1, expand=True)
+    assert P.gathered_length() == 64777                      # 15,625 coarsest entries + 3 levels x 4 x 4,096
+    assert abs(P.gathered_length() - g["gathered_about"]) < 0.01 * g["gathered_about"]
+    assert O.Params(1, 8, 1 << 20, 128, 4, 4, 4096, 32, expand=True).gathered_length() == 65536
+
+
+def _expand_case(rng, N=1024, d=8, L=3, p=4, k=8, C=2):
+    kx = rand_bf16(rng, (N, d))
+    Pe = O.Params(1, 1, N, d, L, p, k, C, expand=True)
+    Pp = O.Params(1, 1, N, d, L + 1, p, k, C)                # one level more: level L-1 is ranked, not kept whole
+    return kx, Pe, Pp
+
+
+@pytest.mark.parametrize("L,p,k,C", [(3, 4, 8, 2), (4, 2, 16, 4), (2, 4, 16, 4), (3, 2, 64, 1)])
+def test_expand_selection_is_the_children_of_the_per_level_selection_one_level_up(L, p, k, C):
+    """The parents the variant picks at level lev+1 are exactly what the per-level reading picks at that level
+    (same scores, chunks and k), given one more level so that level L-1 is ranked too."""
+    rng = np.random.default_rng(L * 100 + p * 10 + C)
+    N = p ** L * 16
+    kx, Pe, Pp = _expand_case(rng, N=N, L=L, p=p, k=k, C=C)
+    Pe.validate()
+    Pp.validate()
+    sel_e = O.select(O.norm_scores(O.pyramid(kx, Pe), Pe), Pe)
+    sel_p = O.select(O.norm_scores(O.pyramid(kx, Pp), Pp), Pp)
+    for lev in range(L - 1):
+        parents = sel_p[lev + 1]
+        want = sorted(int(J) * p + c for J in parents for c in range(p))
+        assert sel_e[lev].tolist() == want, lev
+        assert len(sel_e[lev]) == Pe.picks(lev)
+    assert sel_e[L - 1].tolist() == list(range(Pe.level_size(L - 1)))
+
+
+def test_expand_selection_comes_in_sibling_groups_with_equal_counts_per_chunk():
+    rng = np.random.default_rng(5)
+    P = O.Params(1, 1, 2048, 8, 4, 2, 32, 4, expand=True)
+    scores = [rng.random(P.level_size(lev)).astype(np.float32) for lev in P.scored_levels()]
+    sel = O.select(scores, P)
+    for lev in range(P.L - 1):
+        chosen = set(sel[lev].tolist())
+        assert all((j ^ 1) in chosen for j in chosen)        # p = 2: every entry with its sibling
+        n_c = P.level_size(lev) // P.C
+        counts = np.bincount(sel[lev] // n_c, minlength=P.C)
+        assert np.all(counts == P.picks(lev) // P.C)
+        # brute force: the parents are the top (k/C) of each chunk of level lev+1 by (score desc, index asc)
+        par = scores[lev]                                   # scored level lev+1 is entry lev of the list
+        m, pc = P.parent_picks(lev + 1) // P.C, P.level_size(lev + 1) // P.C
+        want = []
+        for c in range(P.C):
+            js = sorted(range(c * pc, (c + 1) * pc), key=lambda j: (-float(par[j]), j))[:m]
+            want += [2 * j + e for j in sorted(js) for e in range(2)]
+        assert sel[lev].tolist() == want
+
+
+def test_expand_with_k_covering_every_parent_level_is_the_whole_pyramid():
+    rng = np.random.default_rng(9)
+    N, d = 256, 8
+    q, k, v = (rand_bf16(rng, (N, d)) for _ in range(3))
+    Pe = O.Params(1, 1, N, d, 3, 4, 64, 2, expand=True)       # N_1 = 64 = k: every level whole
+    Pw = O.Params(1, 1, N, d, 3, 4, 256, 2)                   # per-level reading with k = N: every level whole
+    assert Pe.gathered_length() == Pw.gathered_length() == 256 + 64 + 16
+    fe, fw = O.forward_head(q, k, v, Pe), O.forward_head(q, k, v, Pw)
+    assert np.array_equal(fe["idx_g"], fw["idx_g"])
+    _close(fe["out"], fw["out"], tol=0)
+
+
+# ----------------------------------------------------------------------------------------------------------------
 # Attention and the whole layer
 # ----------------------------------------------------------------------------------------------------------------
 
