@@ -202,6 +202,22 @@ int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh
   return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
 }
 
+int make_tmap_f16_4d(CUtensorMap* map, const void* base, int d, int rows, int bh, int blocks, uint64_t block_stride,
+                     int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LH_ERR_CUDA;
+  const uint64_t plain = (uint64_t)rows * d * 2 * bh;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)bh, (cuuint64_t)blocks};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2,
+                                 (cuuint64_t)(blocks > 1 ? block_stride : ((plain + 15) & ~uint64_t(15)))};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
+}
+
 }  // namespace lh
 
 using namespace lh;
@@ -369,7 +385,7 @@ int lh_attend(const lh_params* P, const void* qg, const void* kg, const void* vg
   LH_TRY(prepare(P, &dm));
   if (!aligned16(qg) || !aligned16(kg) || !aligned16(vg) || !aligned16(og) || !aligned16(lse))
     return LH_ERR_INVALID_ARG;
-  return launch_attn_fwd(qg, kg, vg, og, lse, dm, (cudaStream_t)stream);
+  return launch_attn_fwd(qg, kv_plain(kg, vg), og, lse, dm, (cudaStream_t)stream);
 }
 
 int lh_scatter(const lh_params* P, const float* og, const int32_t* slot, void* o, void* stream) {
@@ -379,21 +395,15 @@ int lh_scatter(const lh_params* P, const float* og, const int32_t* slot, void* o
   return launch_scatter(og, slot, o, dm, (cudaStream_t)stream);
 }
 
-int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, void* o, void* ctx, void* ws,
-               size_t ws_bytes, void* stream) {
-  LhDims dm;
-  LH_TRY(prepare(P, &dm));
-  cudaStream_t st = (cudaStream_t)stream;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ctx))
-    return LH_ERR_INVALID_ARG;
-  const WsLayout w = ws_layout(dm);
-  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
-  const CtxLayout c = ctx_layout(dm);
-  uint8_t* cb = static_cast<uint8_t*>(ctx);
-  uint8_t* wsb = static_cast<uint8_t*>(ws);
+}  // extern "C"
+
+namespace {
+
+// Steps 1-4a of the forward (pool, score, top-K, order, gather) into the context.
+int forward_select(const LhDims& dm, const void* q, const void* k, const void* v, uint8_t* cb, const CtxLayout& c,
+                   uint8_t* wsb, const WsLayout& w, cudaStream_t st) {
   const void* xs[3] = {q, k, v};
   const int top = dm.L - 1;
-
   // 1-2: pool Q, K, V in one launch; only the coarsest level is stored, plus the key scores
   if (dm.L >= 2) {
     PoolJobs pj;
@@ -426,12 +436,47 @@ int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, 
     gj.job[i].row_off[top] = 0;
     gj.job[i].out = cb + outs[i];
   }
-  LH_TRY(launch_gather(gj, 3, idx_g, dm, st));
+  return launch_gather(gj, 3, idx_g, dm, st);
+}
+
+// The backward's steps before the attention: dO_g window sums (plus, under context parallelism, the next rank's
+// part of the last windows), the per-head scale, fp16 dO_g, D, and the zeroed dQ accumulator.
+int backward_prep(const LhDims& dm, const void* dout, const uint8_t* cb, const CtxLayout& c, uint8_t* wsb,
+                  const WsLayout& w, const float* halo_next, cudaStream_t st) {
+  const int32_t* idx_g = reinterpret_cast<const int32_t*>(cb + c.idx_g);
+  float* dog = reinterpret_cast<float*>(wsb + w.dog);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(wsb + w.amax);
+  if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
+  LH_TRY(launch_scatter_bwd(dout, idx_g, dog, amax, dm, st));
+  if (halo_next)
+    LH_TRY(launch_dog_halo(dog, reinterpret_cast<const int32_t*>(cb + c.slot), halo_next, amax, dm, st));
+  return launch_bwd_prep(dog, reinterpret_cast<const float*>(cb + c.og), amax, wsb + w.dog16,
+                         reinterpret_cast<float*>(wsb + w.dvec), reinterpret_cast<float*>(wsb + w.dinv),
+                         reinterpret_cast<float*>(wsb + w.dqacc), dm, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lh_forward(const lh_params* P, const void* q, const void* k, const void* v, void* o, void* ctx, void* ws,
+               size_t ws_bytes, void* stream) {
+  LhDims dm;
+  LH_TRY(prepare(P, &dm));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ctx))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  const CtxLayout c = ctx_layout(dm);
+  uint8_t* cb = static_cast<uint8_t*>(ctx);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  LH_TRY(forward_select(dm, q, k, v, cb, c, wsb, w, st));
   // 4b: attention over the gathered sequence
   float* og = reinterpret_cast<float*>(cb + c.og);
-  LH_TRY(launch_attn_fwd(cb + c.qg, cb + c.kg, cb + c.vg, og, reinterpret_cast<float*>(cb + c.lse), dm, st));
+  LH_TRY(launch_attn_fwd(cb + c.qg, kv_plain(cb + c.kg, cb + c.vg), og, reinterpret_cast<float*>(cb + c.lse), dm, st));
   // 5: scatter back
-  return launch_scatter(og, slot, o, dm, st);
+  return launch_scatter(og, reinterpret_cast<const int32_t*>(cb + c.slot), o, dm, st);
 }
 
 int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq, void* dk, void* dv, void* ws,
@@ -446,22 +491,14 @@ int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq,
   const CtxLayout c = ctx_layout(dm);
   const uint8_t* cb = static_cast<const uint8_t*>(ctx);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  const int32_t* idx_g = reinterpret_cast<const int32_t*>(cb + c.idx_g);
-  const int32_t* slot = reinterpret_cast<const int32_t*>(cb + c.slot);
-  float* dog = reinterpret_cast<float*>(wsb + w.dog);
-  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
-  float* dinv = reinterpret_cast<float*>(wsb + w.dinv);
+  LH_TRY(backward_prep(dm, dout, cb, c, wsb, w, nullptr, st));
   float* dqacc = reinterpret_cast<float*>(wsb + w.dqacc);
   float* dkg = reinterpret_cast<float*>(wsb + w.dkg);
   float* dvg = reinterpret_cast<float*>(wsb + w.dvg);
-  unsigned int* amax = reinterpret_cast<unsigned int*>(wsb + w.amax);
-  if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
-  LH_TRY(launch_scatter_bwd(dout, idx_g, dog, amax, dm, st));
-  LH_TRY(launch_bwd_prep(dog, reinterpret_cast<const float*>(cb + c.og), amax, wsb + w.dog16, dvec, dinv, dqacc, dm,
-                         st));
-  LH_TRY(launch_attn_bwd(cb + c.qg, cb + c.kg, cb + c.vg, wsb + w.dog16, reinterpret_cast<const float*>(cb + c.lse),
-                         dvec, dinv, dqacc, dkg, dvg, dm, st));
-  return launch_unpool_bwd(dqacc, dkg, dvg, slot, dq, dk, dv, dm, st);
+  LH_TRY(launch_attn_bwd(cb + c.qg, kv_plain(cb + c.kg, cb + c.vg), wsb + w.dog16,
+                         reinterpret_cast<const float*>(cb + c.lse), reinterpret_cast<const float*>(wsb + w.dvec),
+                         reinterpret_cast<const float*>(wsb + w.dinv), dqacc, dkg, dvg, 0, dm, st));
+  return launch_unpool_bwd(dqacc, dkg, dvg, reinterpret_cast<const int32_t*>(cb + c.slot), dq, dk, dv, dm, st);
 }
 
 int lh_scatter_bwd(const lh_params* P, const void* dout, const int32_t* idx_g, float* dog, void* stream) {
@@ -489,7 +526,7 @@ int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void
   if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
   LH_TRY(launch_absmax(dog, amax, dm, st));
   LH_TRY(launch_bwd_prep(dog, og, amax, wsb + w.dog16, dvec, dinv, dqg, dm, st));
-  return launch_attn_bwd(qg, kg, vg, wsb + w.dog16, lse, dvec, dinv, dqg, dkg, dvg, dm, st);
+  return launch_attn_bwd(qg, kv_plain(kg, vg), wsb + w.dog16, lse, dvec, dinv, dqg, dkg, dvg, 0, dm, st);
 }
 
 int lh_set_wait_limit_ns(uint64_t ns) {
@@ -582,3 +619,169 @@ extern "C" int lh_score_topk_static(const lh_params* P, const void* k, const flo
   LH_TRY(launch_topk(scores, sel, slot, dm, st));
   return launch_order(sel, idx_g, slot, dm, st);
 }
+
+// ------------------------------------------------------------------------------------------------------------
+// Context parallelism: the sequence split into G equal shards at chunk boundaries, one per rank.
+// ------------------------------------------------------------------------------------------------------------
+
+namespace lh {
+namespace {
+
+// The shard's parameters and the checks that make the split exact: G | C and G | k keep every chunk, and therefore
+// every pick, inside one shard (each rank selects exactly the global selection's entries of its tokens, S/G of
+// them); the gathered rows per rank must fill whole 128-row attention tiles when G > 1.
+int cp_local(const lh_params* P, int G, int rank, LhDims* glob, LhDims* loc, lh_params* Ploc) {
+  if (!P || G < 1 || rank < 0 || rank >= G) return LH_ERR_INVALID_ARG;
+  LH_TRY(make_dims(P, glob));
+  if (P->C % G || P->k % G || P->N % G) return LH_ERR_INVALID_ARG;
+  *Ploc = *P;
+  Ploc->N = P->N / G;
+  Ploc->k = P->k / G;
+  Ploc->C = P->C / G;
+  LH_TRY(make_dims(Ploc, loc));
+  if ((int64_t)loc->S * G != glob->S) return LH_ERR_INVALID_ARG;  // unreachable when the checks above hold
+  if (G > 1 && loc->S % 128 != 0) return LH_ERR_UNSUPPORTED;
+  return LH_OK;
+}
+
+// cp_local plus the device status word (device entry points only).
+int cp_prepare(const lh_params* P, int G, int rank, LhDims* glob, LhDims* loc, lh_params* Ploc) {
+  LH_TRY(cp_local(P, G, rank, glob, loc, Ploc));
+  return status_ptr(&loc->status);
+}
+
+struct CpSizes {
+  size_t kv_offset, kv_bytes, v_offset, halo_bytes, dkv_bytes;
+};
+CpSizes cp_sizes(const LhDims& loc) {
+  const CtxLayout c = ctx_layout(loc);
+  const size_t rows = (size_t)loc.BH * loc.S * loc.d;
+  CpSizes z;
+  z.kv_offset = c.kg;
+  z.v_offset = c.vg - c.kg;
+  z.kv_bytes = align_up(z.v_offset + rows * 2);
+  z.halo_bytes = (size_t)loc.BH * loc.L * loc.d * 4;
+  z.dkv_bytes = 2 * rows * 4;
+  return z;
+}
+
+}  // namespace
+}  // namespace lh
+
+extern "C" {
+
+int lh_cp_layout(const lh_params* P, int G, lh_cp_layout_t* out) {
+  LhDims glob, loc;
+  lh_params Ploc;
+  if (!out) return LH_ERR_INVALID_ARG;
+  LH_TRY(cp_local(P, G, 0, &glob, &loc, &Ploc));
+  const CpSizes z = cp_sizes(loc);
+  out->local = Ploc;
+  out->S_local = loc.S;
+  out->kv_offset = z.kv_offset;
+  out->kv_bytes = z.kv_bytes;
+  out->v_offset = z.v_offset;
+  out->halo_bytes = z.halo_bytes;
+  out->dkv_bytes = z.dkv_bytes;
+  return LH_OK;
+}
+
+int lh_cp_forward_select(const lh_params* P, int G, int rank, const void* q, const void* k, const void* v, void* ctx,
+                         void* ws, size_t ws_bytes, void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(ctx)) return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  return forward_select(dm, q, k, v, static_cast<uint8_t*>(ctx), ctx_layout(dm), static_cast<uint8_t*>(ws), w,
+                        (cudaStream_t)stream);
+}
+
+int lh_cp_forward_attend(const lh_params* P, int G, int rank, void* ctx, const void* kv_all, float* halo_out,
+                         void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(ctx) || !aligned16(kv_all) || !aligned16(halo_out)) return LH_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const CtxLayout c = ctx_layout(dm);
+  const CpSizes z = cp_sizes(dm);
+  uint8_t* cb = static_cast<uint8_t*>(ctx);
+  const uint8_t* kv = static_cast<const uint8_t*>(kv_all);
+  const KvSource src{kv, kv + z.v_offset, G, (uint64_t)z.kv_bytes, rank * dm.S};
+  float* og = reinterpret_cast<float*>(cb + c.og);
+  LH_TRY(launch_attn_fwd(cb + c.qg, src, og, reinterpret_cast<float*>(cb + c.lse), dm, st));
+  return launch_halo_fwd(og, reinterpret_cast<const int32_t*>(cb + c.slot), halo_out, dm, st);
+}
+
+int lh_cp_forward_scatter(const lh_params* P, int G, int rank, const void* ctx, const float* halo_prev, void* o,
+                          void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(ctx) || !aligned16(o) || (rank > 0 && !aligned16(halo_prev))) return LH_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const CtxLayout c = ctx_layout(dm);
+  const uint8_t* cb = static_cast<const uint8_t*>(ctx);
+  const float* og = reinterpret_cast<const float*>(cb + c.og);
+  const int32_t* slot = reinterpret_cast<const int32_t*>(cb + c.slot);
+  LH_TRY(launch_scatter(og, slot, o, dm, st));
+  return rank > 0 ? launch_scatter_halo(og, slot, halo_prev, o, dm, st) : LH_OK;
+}
+
+int lh_cp_backward_halo(const lh_params* P, int G, int rank, const void* dout, float* halo_out, void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(dout) || !aligned16(halo_out)) return LH_ERR_INVALID_ARG;
+  return launch_halo_bwd(dout, halo_out, dm, (cudaStream_t)stream);
+}
+
+int lh_cp_backward_attend(const lh_params* P, int G, int rank, const void* dout, const void* ctx, const void* kv_all,
+                          const float* halo_next, float* dkv_part, void* ws, size_t ws_bytes, void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(dout) || !aligned16(ctx) || !aligned16(kv_all) || !aligned16(dkv_part) ||
+      (rank < G - 1 && !aligned16(halo_next)))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const CtxLayout c = ctx_layout(dm);
+  const CpSizes z = cp_sizes(dm);
+  const uint8_t* cb = static_cast<const uint8_t*>(ctx);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  LH_TRY(backward_prep(dm, dout, cb, c, wsb, w, rank < G - 1 ? halo_next : nullptr, st));
+  // blocks of ranks after this one see none of its queries: their share of the exchange is zero
+  const size_t block_floats = z.dkv_bytes / 4;
+  if (rank < G - 1 &&
+      cudaMemsetAsync(dkv_part + (rank + 1) * block_floats, 0, (G - 1 - rank) * z.dkv_bytes, st) != cudaSuccess)
+    return LH_ERR_CUDA;
+  const uint8_t* kv = static_cast<const uint8_t*>(kv_all);
+  const KvSource src{kv, kv + z.v_offset, G, (uint64_t)z.kv_bytes, rank * dm.S};
+  const size_t rows = (size_t)dm.BH * dm.S * dm.d;
+  return launch_attn_bwd(cb + c.qg, src, wsb + w.dog16, reinterpret_cast<const float*>(cb + c.lse),
+                         reinterpret_cast<const float*>(wsb + w.dvec), reinterpret_cast<const float*>(wsb + w.dinv),
+                         reinterpret_cast<float*>(wsb + w.dqacc), dkv_part, dkv_part + rows, block_floats, dm, st);
+}
+
+int lh_cp_backward_unpool(const lh_params* P, int G, int rank, const void* ctx, const float* dkv, void* dq, void* dk,
+                          void* dv, void* ws, size_t ws_bytes, void* stream) {
+  LhDims glob, dm;
+  lh_params Ploc;
+  LH_TRY(cp_prepare(P, G, rank, &glob, &dm, &Ploc));
+  if (!aligned16(ctx) || !aligned16(dkv) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return LH_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(dm);
+  if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
+  const CtxLayout c = ctx_layout(dm);
+  const uint8_t* cb = static_cast<const uint8_t*>(ctx);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const size_t rows = (size_t)dm.BH * dm.S * dm.d;
+  return launch_unpool_bwd(reinterpret_cast<const float*>(wsb + w.dqacc), dkv, dkv + rows,
+                           reinterpret_cast<const int32_t*>(cb + c.slot), dq, dk, dv, dm, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
                     const float* __restrict__ dvec, const float* __restrict__ dinv, float* __restrict__ dkg,
-                    float* __restrict__ dvg, int S, float scale, int* status) {
+                    float* __restrict__ dvg, uint64_t dkv_block_stride, int S, int q_off, int kv_tpb, float scale,
+                    int* status) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
@@ -72,10 +73,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // key tiles are numbered globally (tile kt is tile kt % kv_tpb of block kt / kv_tpb); the S local query rows are
+  // global rows q_off .. q_off + S - 1 (q_off = 0 without context parallelism, else a multiple of 128)
   const int kt = blockIdx.x;  // key tile: tile 0 meets the most query sub-tiles and is scheduled first
   const int bh = blockIdx.y;
+  const int kblk = kt / kv_tpb, krow0 = (kt % kv_tpb) * kKTile;  // block of the key tile and its first row there
   const int nq = (S + kQTile - 1) / kQTile;
-  const int i0 = 2 * kt;  // first sub-tile with a query at or after the tile's first key
+  const int i0 = max(0, 2 * kt - q_off / kQTile);  // first local sub-tile with a query at or after the tile's first key
   const int nit = nq - i0;
   const float scale_log2 = scale * kLog2e;
   const float inv_scale = dinv[bh];
@@ -117,8 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       mbar_arrive_expect_tx(bar(Lay::B_KV), 2 * Lay::KT);
       for (int db = 0; db < D / 64; ++db) {
-        tma_load_3d(sb + Lay::K + db * 16384, &tmK, bar(Lay::B_KV), db * 64, kt * kKTile, bh);
-        tma_load_3d(sb + Lay::V + db * 16384, &tmV, bar(Lay::B_KV), db * 64, kt * kKTile, bh);
+        tma_load_4d(sb + Lay::K + db * 16384, &tmK, bar(Lay::B_KV), db * 64, krow0, bh, kblk);
+        tma_load_4d(sb + Lay::V + db * 16384, &tmV, bar(Lay::B_KV), db * 64, krow0, bh, kblk);
       }
       for (int it = 0; it < nit && ok; ++it) {
         const int s = it % kStages;
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;  // key row inside the tile = TMEM lane
     const int ct = threadIdx.x - 64;    // 0..127 inside the compute group
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int key = kt * kKTile + r;
+    const int key = kt * kKTile + r;  // global key row
     float* s_lse = reinterpret_cast<float*>(smem + Lay::STAT);
     float* s_d = s_lse + 2 * kQTile;
     bool ok = true;
@@ -231,7 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t pk[32], dk[32];
       if (ok) {
-        const bool diag = i * kQTile < key;  // some query of the sub-tile precedes the key (masked)
+        const int qg0 = q_off + i * kQTile;  // global row of the sub-tile's first query
+        const bool diag = qg0 < key;         // some query of the sub-tile precedes the key (masked)
         // dS = P (dP - D) scale = P fma(dP, scale, -D scale); the fp16 range is checked on the packed values (a
         // value beyond it became an infinity, NaN stays NaN): largest |dS| half2 over 4 independent chains
         __half2 hm[4];
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             float pv = ex2(fmaf(sv[c + e], scale_log2, -lv[e]));
-            if (diag && i * kQTile + c + e < key) pv = 0.f;  // query does not see key `key`
+            if (diag && qg0 + c + e < key) pv = 0.f;  // query does not see key `key`
             p2[e] = pv;
             d2[e] = pv * fmaf(dp[c + e], scale, -dv[e]);
           }
@@ -302,8 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           tmem_ld32(tacc + lane_base + c * 32, v);
           tmem_ld_wait();
-          if (key < S) {
-            float4* dst = reinterpret_cast<float4*>(dst_base + ((int64_t)bh * S + key) * D + c * 32);
+          if (krow0 + r < S) {  // the key row exists (the last tile of a single ragged block is partial)
+            float4* dst = reinterpret_cast<float4*>(dst_base + kblk * dkv_block_stride +
+                                                    ((int64_t)bh * S + krow0 + r) * D + c * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
               dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
@@ -361,30 +367,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-int launch_bwd_t(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse, const float* dvec,
-                 const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm, cudaStream_t st) {
+int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
+                 const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride, const LhDims& dm,
+                 cudaStream_t st) {
+  if (kv.q_off % kKTile != 0 || (kv.blocks > 1 && dm.S % kKTile != 0)) return LH_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH, kQTile) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH, kKTile) ||
-      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH, kKTile) || make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH, kQTile) ||
-      make_tmap_f32_3d(&mdq, dqacc, D, dm.S, dm.BH, 32, kQTile))
+  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH, kQTile) ||
+      make_tmap_f16_4d(&mk, kv.k, D, dm.S, dm.BH, kv.blocks, kv.block_stride, kKTile) ||
+      make_tmap_f16_4d(&mv, kv.v, D, dm.S, dm.BH, kv.blocks, kv.block_stride, kKTile) ||
+      make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH, kQTile) || make_tmap_f32_3d(&mdq, dqacc, D, dm.S, dm.BH, 32, kQTile))
     return LH_ERR_CUDA;
   const int smem = BwdLayout<D>::BYTES + 1024;
   if (cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LH_ERR_CUDA;
-  const int nt = (dm.S + kKTile - 1) / kKTile;
+  const int tpb = (dm.S + kKTile - 1) / kKTile;            // key tiles per block
+  const int nt = (kv.q_off + dm.S + kKTile - 1) / kKTile;  // key tiles the local queries see
   KernelTimer timer("attn_bwd", st);
-  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, dvec, dinv, dkg, dvg, dm.S,
+  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, dvec, dinv, dkg, dvg,
+                                                               dkv_block_stride, dm.S, kv.q_off, tpb,
                                                                1.0f / sqrtf((float)D), dm.status);
   return check_launch();
 }
 
 }  // namespace
 
-int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse,
-                    const float* dvec, const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm,
-                    cudaStream_t st) {
-  return dm.d == 64 ? launch_bwd_t<64>(qg, kg, vg, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dm, st)
-                    : launch_bwd_t<128>(qg, kg, vg, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dm, st);
+int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
+                    const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride,
+                    const LhDims& dm, cudaStream_t st) {
+  return dm.d == 64 ? launch_bwd_t<64>(qg, kv, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st)
+                    : launch_bwd_t<128>(qg, kv, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st);
 }
 
 }  // namespace lh

@@ -47,7 +47,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, float* __restrict__ og, float* __restrict__ lse, int S,
-                    int npair, float scale_log2, int* status) {
+                    int npair, int q_tile0, int kv_tpb, float scale_log2, int* status) {
   using Lay = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
@@ -61,7 +61,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.y;
   const int ntile = (S + kTile - 1) / kTile;
   const bool v1 = 2 * pt + 1 < ntile;    // the pair's second query tile exists
-  const int nkv0 = 2 * pt + 1;           // key tiles of query tile 0 (its diagonal is tile 2 pt)
+  // key tiles are numbered globally: the local query tile t is global tile q_tile0 + t (context parallelism puts
+  // the local queries after q_tile0 tiles of earlier ranks' keys); key tile j is tile j % kv_tpb of block j / kv_tpb
+  const int nkv0 = q_tile0 + 2 * pt + 1;  // key tiles of query tile 0 (its diagonal is the last one)
   const int nkv = v1 ? nkv0 + 1 : nkv0;  // key tiles loaded (= those of query tile 1 when it exists)
 
   if (threadIdx.x == 0) {
@@ -105,7 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mbar_arrive_expect_tx(bar(Lay::B_KF + b), Lay::TILE);
         for (int db = 0; db < D / 64; ++db)
-          tma_load_3d(sb + Lay::K + b * Lay::TILE + db * 16384, &tmK, bar(Lay::B_KF + b), db * 64, j * kTile, bh);
+          tma_load_4d(sb + Lay::K + b * Lay::TILE + db * 16384, &tmK, bar(Lay::B_KF + b), db * 64,
+                      (j % kv_tpb) * kTile, bh, j / kv_tpb);
         if (j >= 2) ok = mbar_wait(bar(Lay::B_VE + b), ph, &s_wait, status);
         if (!ok) {
           kv_issued = j;  // K_j in flight without its V
@@ -114,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(bar(Lay::B_VF + b), Lay::TILE);
         for (int db = 0; db < D / 64; ++db)
-          tma_load_3d(sb + Lay::V + b * Lay::TILE + db * 16384, &tmV, bar(Lay::B_VF + b), db * 64, j * kTile, bh);
+          tma_load_4d(sb + Lay::V + b * Lay::TILE + db * 16384, &tmV, bar(Lay::B_VF + b), db * 64,
+                      (j % kv_tpb) * kTile, bh, j / kv_tpb);
         kv_issued = j + 1;
       }
       if (!ok) {  // drain the copies this thread issued before leaving
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
       const uint32_t tS = tmem + 128 * q + lane_base, tO = tmem + 256 + 128 * q + lane_base;
       const int nkv_q = nkv0 + q;
-      const int diag = 2 * pt + q;
+      const int diag = q_tile0 + 2 * pt + q;  // global key tile on the diagonal
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv_q && ok; ++j) {
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         const float inv_l = 1.0f / l_run;
-        const int grow_idx = diag * kTile + row;
+        const int grow_idx = (2 * pt + q) * kTile + row;  // local query row
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -312,11 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-int launch_fwd_t(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
-                 cudaStream_t st) {
+int launch_fwd_t(const void* qg, const KvSource& kv, float* og, float* lse, const LhDims& dm, cudaStream_t st) {
+  if (kv.q_off % kTile != 0 || (kv.blocks > 1 && dm.S % kTile != 0)) return LH_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH) || make_tmap_f16_3d(&mk, kg, D, dm.S, dm.BH) ||
-      make_tmap_f16_3d(&mv, vg, D, dm.S, dm.BH))
+  if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH) ||
+      make_tmap_f16_4d(&mk, kv.k, D, dm.S, dm.BH, kv.blocks, kv.block_stride) ||
+      make_tmap_f16_4d(&mv, kv.v, D, dm.S, dm.BH, kv.blocks, kv.block_stride))
     return LH_ERR_CUDA;
   // at least 120 KB, so that one CTA (and its 512 tensor-memory columns) occupies an SM
   int smem = FwdLayout<D>::BYTES + 1024;
@@ -327,16 +332,15 @@ int launch_fwd_t(const void* qg, const void* kg, const void* vg, float* og, floa
   const int npair = (nt + 1) / 2;
   const float scale_log2 = kLog2e / sqrtf((float)D);
   KernelTimer timer("attn_fwd", st);
-  attn_fwd_kernel<D><<<dim3(npair, dm.BH), kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, npair, scale_log2,
-                                                                  dm.status);
+  attn_fwd_kernel<D><<<dim3(npair, dm.BH), kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, npair, kv.q_off / kTile,
+                                                                  nt, scale_log2, dm.status);
   return check_launch();
 }
 
 }  // namespace
 
-int launch_attn_fwd(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
-                    cudaStream_t st) {
-  return dm.d == 64 ? launch_fwd_t<64>(qg, kg, vg, og, lse, dm, st) : launch_fwd_t<128>(qg, kg, vg, og, lse, dm, st);
+int launch_attn_fwd(const void* qg, const KvSource& kv, float* og, float* lse, const LhDims& dm, cudaStream_t st) {
+  return dm.d == 64 ? launch_fwd_t<64>(qg, kv, og, lse, dm, st) : launch_fwd_t<128>(qg, kv, og, lse, dm, st);
 }
 
 }  // namespace lh

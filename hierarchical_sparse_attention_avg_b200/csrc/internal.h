@@ -54,16 +54,41 @@ int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax,
                     float* dqacc, const LhDims& dm, cudaStream_t st);
 int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st);
-int launch_attn_fwd(const void* qg, const void* kg, const void* vg, float* og, float* lse, const LhDims& dm,
-                    cudaStream_t st);
-// qg, kg, vg, dog16: fp16 [BH, S, d] (dog16 scaled per head); dvec scaled alike; dinv: inverse scales.
-// dqacc (fp32, zeroed) accumulates dQ_g; dkg, dvg (fp32) receive dK_g, dV_g.
-int launch_attn_bwd(const void* qg, const void* kg, const void* vg, const void* dog16, const float* lse,
-                    const float* dvec, const float* dinv, float* dqacc, float* dkg, float* dvg, const LhDims& dm,
+// Keys and values of the attention: `blocks` blocks of dm.S rows each (one per rank of a context-parallel group;
+// a single block otherwise), block g of K at k + g * block_stride bytes (V likewise), each fp16 [BH, S, d].  The
+// queries (dm.S local rows) have global rows q_off .. q_off + S - 1 (q_off a multiple of 128; 0 without context
+// parallelism) and see every key of global row <= their own, i.e. the first q_off + S keys.
+struct KvSource {
+  const void* k;
+  const void* v;
+  int blocks;
+  uint64_t block_stride;
+  int q_off;
+};
+inline KvSource kv_plain(const void* k, const void* v) { return KvSource{k, v, 1, 0, 0}; }
+
+int launch_attn_fwd(const void* qg, const KvSource& kv, float* og, float* lse, const LhDims& dm, cudaStream_t st);
+// qg, dog16: fp16 [BH, S, d] (dog16 scaled per head); dvec scaled alike; dinv: inverse scales.  dqacc (fp32,
+// zeroed) accumulates dQ_g of the local queries; dK_g and dV_g (fp32) of the key rows of block g are written to
+// dkg / dvg + g * dkv_block_stride floats, [BH, S, d] each.
+int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
+                    const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride,
+                    const LhDims& dm, cudaStream_t st);
+
+// Context parallelism: halo rows exchanged between neighbouring ranks (fp32 [BH][L][d], see cp.cu).
+int launch_halo_fwd(const float* og, const int32_t* slot, float* halo, const LhDims& dm, cudaStream_t st);
+int launch_scatter_halo(const float* og, const int32_t* slot, const float* halo, void* o, const LhDims& dm,
+                        cudaStream_t st);
+int launch_halo_bwd(const void* dout, float* halo, const LhDims& dm, cudaStream_t st);
+int launch_dog_halo(float* dog, const int32_t* slot, const float* halo, unsigned int* amax, const LhDims& dm,
                     cudaStream_t st);
 
 // Encode a 3-D fp16 tensor map over [BH][rows][d] with a {64, box_rows, 1} box and 128-byte swizzle.
 int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_rows = 128);
+// Encode a 4-D fp16 tensor map over [blocks][BH][rows][d] (block stride in bytes) with a {64, box_rows, 1, 1} box
+// and 128-byte swizzle.
+int make_tmap_f16_4d(CUtensorMap* map, const void* base, int d, int rows, int bh, int blocks, uint64_t block_stride,
+                     int box_rows = 128);
 // Encode a 3-D fp32 tensor map over [BH][rows][d] with a {box_cols, box_rows, 1} box, no swizzle.
 int make_tmap_f32_3d(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_cols, int box_rows);
 

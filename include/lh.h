@@ -261,6 +261,72 @@ int lh_step_host(const lh_params* P, const void* q, const void* k, const void* v
                  void* dk, void* dv, int heads_per_chunk, void* dev, size_t dev_bytes, void* stream, void* h2d_stream,
                  void* d2h_stream);
 
+/* ---- context parallelism: one sequence split across G ranks ------------------------------------------ */
+
+/* [E] "Може ли този подход да скалира отвъд един GPU по начин, който ops екипите ще приемат?": beyond ~100K tokens
+ * the layer runs context-parallel; pooling, scoring and top-K stay local to each shard and the gathered dense
+ * subsequence takes part in ordinary ring attention.  Here the N tokens of every head are split into G equal
+ * shards, rank r holding tokens [r N/G, (r+1) N/G) of Q, K, V, dO, O, dQ, dK, dV as its own bf16 [B,H,N/G,d]
+ * tensors.  Requirements: G | C and G | k (every chunk, so every pick, lies inside one shard: rank r's selection is
+ * exactly the global selection's entries in its shard, S/G of them, and its gathered rows are rows r S/G ..
+ * (r+1) S/G - 1 of the global gathered sequence); for G > 1 also S/G a multiple of 128 (LH_ERR_UNSUPPORTED
+ * otherwise).  Results equal those of lh_forward / lh_backward on the whole sequence (selection and gathered rows
+ * bit-exact; outputs up to the order of fp32 sums).
+ *
+ * The caller runs the exchanges (NCCL over NVLink, say), each into its own device memory:
+ *   forward:  lh_cp_forward_select -> all-gather of each rank's K_g/V_g chunk (kv_bytes bytes at kv_offset of its
+ *             ctx, rank order) into kv_all -> lh_cp_forward_attend -> all-gather of the halo blocks ->
+ *             lh_cp_forward_scatter with rank r-1's block;
+ *   backward: lh_cp_backward_halo -> all-gather of the halo blocks -> lh_cp_backward_attend with rank r+1's block
+ *             -> reduce-scatter (sum) of dkv_part (G blocks of dkv_bytes, block g to rank g) -> lh_cp_backward_unpool.
+ * ctx and ws are per rank, sized for the shard's parameters (lh_cp_layout(...).local), and ws must keep its
+ * contents from lh_cp_backward_attend to lh_cp_backward_unpool (it holds the dQ_g accumulator). */
+typedef struct lh_cp_layout_t {
+  lh_params local;      /* the shard's parameters: N/G, k/G, C/G, the rest as given */
+  int64_t S_local;      /* gathered rows per rank, S/G */
+  uint64_t kv_offset;   /* byte offset, inside a rank's ctx, of the chunk it contributes to the K_g/V_g exchange */
+  uint64_t kv_bytes;    /* bytes of that chunk (K_g at 0, V_g at v_offset); kv_all holds G chunks in rank order */
+  uint64_t v_offset;    /* byte offset of V_g inside a chunk */
+  uint64_t halo_bytes;  /* bytes of one rank's halo block, fp32 [B*H][L][d]; a halo exchange holds G blocks */
+  uint64_t dkv_bytes;   /* bytes of one block of the dK_g/dV_g exchange, fp32 [2][B*H][S/G][d] (dK_g then dV_g) */
+} lh_cp_layout_t;
+
+/* Sizes of the split for global parameters P over G ranks; LH_OK or the validation error. */
+int lh_cp_layout(const lh_params* P, int G, lh_cp_layout_t* out);
+
+/* Forward steps 1-4a on rank `rank`'s shard: pool, score, top-K, order and gather of its tokens into ctx. */
+int lh_cp_forward_select(const lh_params* P, int G, int rank, const void* q, const void* k, const void* v, void* ctx,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Forward step 4b: the shard's gathered queries (global rows rank*S/G ..) attend causally over the gathered keys
+ * and values of ranks 0..rank in kv_all (G chunks of kv_bytes, as exchanged); O_g and LSE go to ctx.  Then
+ * halo_out (one block, fp32 [B*H][L][d]) receives, per head and level l, O_g of the shard's last level-l entry
+ * (zeros when it is not selected): the next rank's tokens t < p^l - 1 take it at level l. */
+int lh_cp_forward_attend(const lh_params* P, int G, int rank, void* ctx, const void* kv_all, float* halo_out,
+                         void* stream);
+
+/* Forward step 5: the offset scatter-back of the shard's tokens; halo_prev is rank rank-1's halo block (ignored,
+ * may be NULL, on rank 0).  o: bf16 [B,H,N/G,d]. */
+int lh_cp_forward_scatter(const lh_params* P, int G, int rank, const void* ctx, const float* halo_prev, void* o,
+                          void* stream);
+
+/* Backward exchange: halo_out (one block) receives, per head and level l, the fp32 sum of the shard's first p^l - 1
+ * rows of dout: the part of the previous rank's last level-l window that lies in this shard. */
+int lh_cp_backward_halo(const lh_params* P, int G, int rank, const void* dout, float* halo_out, void* stream);
+
+/* Backward through the attention: dO_g window sums of the shard (plus halo_next, rank rank+1's halo block, in the
+ * last window of each level; ignored, may be NULL, on the last rank), then the attention backward of the shard's
+ * queries against the keys of ranks 0..rank.  dQ_g stays in ws; dkv_part (G blocks of dkv_bytes) receives this
+ * rank's contribution to dK_g/dV_g of every rank's keys (zeros for ranks after this one).  dQ_g is accumulated
+ * with fp32 reduce-adds in no fixed order. */
+int lh_cp_backward_attend(const lh_params* P, int G, int rank, const void* dout, const void* ctx, const void* kv_all,
+                          const float* halo_next, float* dkv_part, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward unpool: dq, dk, dv (bf16 [B,H,N/G,d]) of the shard from dQ_g (in ws) and dkv, this rank's block of the
+ * summed exchange (fp32 [2][B*H][S/G][d]). */
+int lh_cp_backward_unpool(const lh_params* P, int G, int rank, const void* ctx, const float* dkv, void* dq, void* dk,
+                          void* dv, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- status ------------------------------------------------------------------------------------------ */
 
 /* Synchronises `stream`, returns the first device-side error recorded since the last call (LH_OK if none)
