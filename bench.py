@@ -130,8 +130,8 @@ def measured_traffic(kernel: str, w: dict):
     if not os.path.exists(TRAFFIC_FILE):
         return None, None
     for line in open(TRAFFIC_FILE):
-        f = line.split()
-        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] in WORKLOADS:
+        f = line.split("#")[0].split()
+        if len(f) == 5 and f[0] == kernel and f[1] in WORKLOADS:
             if f[4] != source_digest(kernel):
                 continue
             got = int(f[2]) + int(f[3])

@@ -106,7 +106,7 @@ struct WsLayout {
   // forward / selection
   size_t scores, coarse[3], sel, fwd_total;
   // backward
-  size_t dog, dog16, dvec, amax, dinv, dqacc, dkg, dvg, bwd_total;
+  size_t dog, dog16, stats, amax, dinv, dqacc, dkg, dvg, bwd_total;
   size_t total;
 };
 WsLayout ws_layout(const LhDims& dm) {
@@ -121,7 +121,7 @@ WsLayout ws_layout(const LhDims& dm) {
   o = 0;
   w.dog = o; o = align_up(o + rows * dm.d * 4);    // fp32 window sums
   w.dog16 = o; o = align_up(o + rows * dm.d * 2);  // fp16, scaled per head
-  w.dvec = o; o = align_up(o + rows * 4);
+  w.stats = o; o = align_up(o + (size_t)dm.BH * stats_stride(dm) * 2 * 4);  // -LSE log2 e, -D / sqrt(d)
   w.amax = o; o = align_up(o + (size_t)dm.BH * 4);
   w.dinv = o; o = align_up(o + (size_t)dm.BH * 4);
   w.dqacc = o; o = align_up(o + rows * dm.d * 4);
@@ -198,6 +198,20 @@ int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
+}
+
+int make_tmap_stats(CUtensorMap* map, const float* stats, int S, int bh, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LH_ERR_CUDA;
+  const uint64_t stride = (uint64_t)((S + 3) & ~3) * 4;
+  const cuuint64_t dims[3] = {(cuuint64_t)S, (cuuint64_t)bh, 2};
+  const cuuint64_t strides[2] = {(cuuint64_t)stride, (cuuint64_t)(stride * bh)};
+  const cuuint32_t box[3] = {(cuuint32_t)box_rows, 1, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(stats), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LH_OK : LH_ERR_CUDA;
 }
@@ -450,9 +464,9 @@ int backward_prep(const LhDims& dm, const void* dout, const uint8_t* cb, const C
   LH_TRY(launch_scatter_bwd(dout, idx_g, dog, amax, dm, st));
   if (halo_next)
     LH_TRY(launch_dog_halo(dog, reinterpret_cast<const int32_t*>(cb + c.slot), halo_next, amax, dm, st));
-  return launch_bwd_prep(dog, reinterpret_cast<const float*>(cb + c.og), amax, wsb + w.dog16,
-                         reinterpret_cast<float*>(wsb + w.dvec), reinterpret_cast<float*>(wsb + w.dinv),
-                         reinterpret_cast<float*>(wsb + w.dqacc), dm, st);
+  return launch_bwd_prep(dog, reinterpret_cast<const float*>(cb + c.og), reinterpret_cast<const float*>(cb + c.lse),
+                         amax, wsb + w.dog16, reinterpret_cast<float*>(wsb + w.stats),
+                         reinterpret_cast<float*>(wsb + w.dinv), reinterpret_cast<float*>(wsb + w.dqacc), dm, st);
 }
 
 }  // namespace
@@ -496,8 +510,8 @@ int lh_backward(const lh_params* P, const void* dout, const void* ctx, void* dq,
   float* dkg = reinterpret_cast<float*>(wsb + w.dkg);
   float* dvg = reinterpret_cast<float*>(wsb + w.dvg);
   LH_TRY(launch_attn_bwd(cb + c.qg, kv_plain(cb + c.kg, cb + c.vg), wsb + w.dog16,
-                         reinterpret_cast<const float*>(cb + c.lse), reinterpret_cast<const float*>(wsb + w.dvec),
-                         reinterpret_cast<const float*>(wsb + w.dinv), dqacc, dkg, dvg, 0, dm, st));
+                         reinterpret_cast<const float*>(wsb + w.stats), reinterpret_cast<const float*>(wsb + w.dinv),
+                         dqacc, dkg, dvg, 0, dm, st));
   return launch_unpool_bwd(dqacc, dkg, dvg, reinterpret_cast<const int32_t*>(cb + c.slot), dq, dk, dv, dm, st);
 }
 
@@ -520,13 +534,13 @@ int lh_attend_bwd(const lh_params* P, const void* qg, const void* kg, const void
   const WsLayout w = ws_layout(dm);
   if (!aligned16(ws) || ws_bytes < w.total) return ws ? LH_ERR_WORKSPACE : LH_ERR_INVALID_ARG;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  float* stats = reinterpret_cast<float*>(wsb + w.stats);
   float* dinv = reinterpret_cast<float*>(wsb + w.dinv);
   unsigned int* amax = reinterpret_cast<unsigned int*>(wsb + w.amax);
   if (cudaMemsetAsync(amax, 0, (size_t)dm.BH * 4, st) != cudaSuccess) return LH_ERR_CUDA;
   LH_TRY(launch_absmax(dog, amax, dm, st));
-  LH_TRY(launch_bwd_prep(dog, og, amax, wsb + w.dog16, dvec, dinv, dqg, dm, st));
-  return launch_attn_bwd(qg, kv_plain(kg, vg), wsb + w.dog16, lse, dvec, dinv, dqg, dkg, dvg, 0, dm, st);
+  LH_TRY(launch_bwd_prep(dog, og, lse, amax, wsb + w.dog16, stats, dinv, dqg, dm, st));
+  return launch_attn_bwd(qg, kv_plain(kg, vg), wsb + w.dog16, stats, dinv, dqg, dkg, dvg, 0, dm, st);
 }
 
 int lh_set_wait_limit_ns(uint64_t ns) {
@@ -762,9 +776,9 @@ int lh_cp_backward_attend(const lh_params* P, int G, int rank, const void* dout,
   const uint8_t* kv = static_cast<const uint8_t*>(kv_all);
   const KvSource src{kv, kv + z.v_offset, G, (uint64_t)z.kv_bytes, rank * dm.S};
   const size_t rows = (size_t)dm.BH * dm.S * dm.d;
-  return launch_attn_bwd(cb + c.qg, src, wsb + w.dog16, reinterpret_cast<const float*>(cb + c.lse),
-                         reinterpret_cast<const float*>(wsb + w.dvec), reinterpret_cast<const float*>(wsb + w.dinv),
-                         reinterpret_cast<float*>(wsb + w.dqacc), dkv_part, dkv_part + rows, block_floats, dm, st);
+  return launch_attn_bwd(cb + c.qg, src, wsb + w.dog16, reinterpret_cast<const float*>(wsb + w.stats),
+                         reinterpret_cast<const float*>(wsb + w.dinv), reinterpret_cast<float*>(wsb + w.dqacc),
+                         dkv_part, dkv_part + rows, block_floats, dm, st);
 }
 
 int lh_cp_backward_unpool(const lh_params* P, int G, int rank, const void* ctx, const float* dkv, void* dq, void* dk,

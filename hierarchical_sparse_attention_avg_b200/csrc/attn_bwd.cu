@@ -48,8 +48,9 @@ struct BwdLayout {
   static constexpr uint32_t DO = Q + kStages * QT;           // kStages
   static constexpr uint32_t DS = DO + kStages * QT;          // 2 buffers (dS^T, the B operand of dQ^T)
   static constexpr uint32_t DQ = DS + 2 * PT;                // staging: [d/32][64 q][32 f] fp32
-  static constexpr uint32_t STAT = DQ + kQTile * D * 4;      // [2][64] LSE*log2e, [2][64] D
-  static constexpr uint32_t BAR = STAT + 4 * kQTile * 4;
+  static constexpr uint32_t ST = 2 * kQTile * 4;             // one stage's statistics: [2][64] fp32
+  static constexpr uint32_t STAT = DQ + kQTile * D * 4;      // kStages x {-LSE log2 e, -D/sqrt(d)} of the sub-tile
+  static constexpr uint32_t BAR = STAT + kStages * ST;
   static constexpr uint32_t B_KV = 0, B_QF = 1, B_QE = 1 + kStages, B_SF = 1 + 2 * kStages, B_DSF = B_SF + 2,
                             B_MM = B_DSF + 2, B_DQF = B_MM + 2, B_FIN = B_DQF + 2, B_DRAIN = B_FIN + 1,
                             NBAR = B_DRAIN + 1;
@@ -60,8 +61,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
-                    const float* __restrict__ dvec, const float* __restrict__ dinv, float* __restrict__ dkg,
+                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmST,
+                    const float* __restrict__ dinv, float* __restrict__ dkg,
                     float* __restrict__ dvg, uint64_t dkv_block_stride, int S, int q_off, int kv_tpb, float scale,
                     int* status) {
   using Lay = BwdLayout<D>;
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmDO);
     prefetch_tmap(&tmDQ);
+    prefetch_tmap(&tmST);
   }
   if (warp == 1) tmem_alloc(smem_u32(&s_tmem), 512);
   tc_fence_before();
@@ -129,11 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it >= kStages) ok = mbar_wait(bar(Lay::B_QE + s), ((it / kStages) - 1) & 1, &s_wait, status);
         if (!ok) break;
         const int row = (i0 + it) * kQTile;
-        mbar_arrive_expect_tx(bar(Lay::B_QF + s), 2 * Lay::QT);
+        mbar_arrive_expect_tx(bar(Lay::B_QF + s), 2 * Lay::QT + Lay::ST);
         for (int db = 0; db < D / 64; ++db) {
           tma_load_3d(sb + Lay::Q + s * Lay::QT + db * 8192, &tmQ, bar(Lay::B_QF + s), db * 64, row, bh);
           tma_load_3d(sb + Lay::DO + s * Lay::QT + db * 8192, &tmDO, bar(Lay::B_QF + s), db * 64, row, bh);
         }
+        tma_load_3d(sb + Lay::STAT + s * Lay::ST, &tmST, bar(Lay::B_QF + s), row, bh, 0);  // both planes
         issued = it + 1;
       }
       if (!ok) {
@@ -199,69 +202,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- compute: P^T and dS^T rows
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row inside the tile = TMEM lane
-    const int ct = threadIdx.x - 64;    // 0..127 inside the compute group
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int key = kt * kKTile + r;  // global key row
-    float* s_lse = reinterpret_cast<float*>(smem + Lay::STAT);
-    float* s_d = s_lse + 2 * kQTile;
     bool ok = true;
-    // statistics (LSE and D) of one query each, loaded one sub-tile ahead so that their latency is hidden
-    auto load_stats = [&](int i, float& l, float& dd) {
-      const int q = i * kQTile + ct;
-      l = (ct < kQTile && q < S) ? lse[(int64_t)bh * S + q] * kLog2e : INFINITY;
-      dd = (ct < kQTile && q < S) ? dvec[(int64_t)bh * S + q] * scale : 0.f;  // D already times the scale
-    };
-    float nl = INFINITY, nd = 0.f;
-    if (nit > 0) load_stats(i0, nl, nd);
-    for (int it = 0; it < nit; ++it) {
-      const int b = it & 1, i = i0 + it;
-      // statistics of the sub-tile into buffer b (its previous readers, sub-tile it-2, are done: same threads)
-      if (ct < kQTile) {
-        s_lse[b * kQTile + ct] = nl;
-        s_d[b * kQTile + ct] = nd;
-      }
-      if (it + 1 < nit) load_stats(i + 1, nl, nd);
-      ok = named_barrier_and(kBarCompute, 128, ok);
-      if (!ok) break;
+    const uint64_t scl2 = f2pack(scale_log2, scale_log2), sc2 = f2pack(scale, scale);
+    for (int it = 0; it < nit && ok; ++it) {
+      const int b = it & 1, s = it % kStages, i = i0 + it;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_wait, status));
+      // the sub-tile's statistics arrived with its Q/dO stage (complete before S^T was issued)
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QF + s), (it / kStages) & 1, &s_wait, status));
+      if (!ok) break;
       float sv[64], dp[64];
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(tmem + 128 * b + lane_base, *reinterpret_cast<float(*)[32]>(&sv[0]));
-        tmem_ld32(tmem + 128 * b + lane_base + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
-        tmem_ld32(tmem + 128 * b + 64 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[0]));
-        tmem_ld32(tmem + 128 * b + 96 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[32]));
-        tmem_ld_wait();
-      }
+      tc_fence_after();
+      tmem_ld32(tmem + 128 * b + lane_base, *reinterpret_cast<float(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + 128 * b + lane_base + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+      tmem_ld32(tmem + 128 * b + 64 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[0]));
+      tmem_ld32(tmem + 128 * b + 96 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[32]));
+      tmem_ld_wait();
       uint32_t pk[32], dk[32];
-      if (ok) {
+      {
         const int qg0 = q_off + i * kQTile;  // global row of the sub-tile's first query
         const bool diag = qg0 < key;         // some query of the sub-tile precedes the key (masked)
-        // dS = P (dP - D) scale = P fma(dP, scale, -D scale); the fp16 range is checked on the packed values (a
-        // value beyond it became an infinity, NaN stays NaN): largest |dS| half2 over 4 independent chains
+        // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D) scale = P fma(dP, scale, -D scale), two columns per
+        // packed fp32x2 instruction; the statistics are stored negated, as 16-byte broadcast vectors.  The fp16
+        // range of dS is checked on the packed values (beyond it: an infinity; NaN stays NaN): largest |dS| half2
+        // over 4 independent chains
         __half2 hm[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) hm[k] = __float2half2_rn(0.f);
-        // the sub-tile's statistics as 16-byte vectors (the same for every thread: broadcast loads)
-        const float4* sl4 = reinterpret_cast<const float4*>(s_lse + b * kQTile);
-        const float4* sd4 = reinterpret_cast<const float4*>(s_d + b * kQTile);
+        const ulonglong2* nl4 = reinterpret_cast<const ulonglong2*>(smem + Lay::STAT + s * Lay::ST);
+        const ulonglong2* nd4 = nl4 + kQTile / 4;
 #pragma unroll
-        for (int c = 0; c < kQTile; c += 2) {
-          float p2[2], d2[2];
-          const float4 l4 = sl4[c >> 2], d4 = sd4[c >> 2];
-          const float lv[2] = {(c & 2) ? l4.z : l4.x, (c & 2) ? l4.w : l4.y};
-          const float dv[2] = {(c & 2) ? d4.z : d4.x, (c & 2) ? d4.w : d4.y};
+        for (int c = 0; c < kQTile; c += 4) {
+          const ulonglong2 nl = nl4[c >> 2], nd = nd4[c >> 2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float pv = ex2(fmaf(sv[c + e], scale_log2, -lv[e]));
-            if (diag && qg0 + c + e < key) pv = 0.f;  // query does not see key `key`
-            p2[e] = pv;
-            d2[e] = pv * fmaf(dp[c + e], scale, -dv[e]);
+          for (int h = 0; h < 2; ++h) {
+            const int cc = c + 2 * h;
+            const uint64_t arg = fma_f32x2(f2pack(sv[cc], sv[cc + 1]), scl2, h ? nl.y : nl.x);
+            float p0 = ex2(f2lo(arg)), p1 = ex2(f2hi(arg));
+            if (diag) {  // queries that precede the key do not see it
+              if (qg0 + cc < key) p0 = 0.f;
+              if (qg0 + cc + 1 < key) p1 = 0.f;
+            }
+            const uint64_t p2 = f2pack(p0, p1);
+            const uint64_t d2 = mul_f32x2(p2, fma_f32x2(f2pack(dp[cc], dp[cc + 1]), sc2, h ? nd.y : nd.x));
+            pk[cc / 2] = pack_half2_rn(p0, p1);
+            dk[cc / 2] = pack_half2_rn(f2lo(d2), f2hi(d2));
+            const __half2 hv = *reinterpret_cast<const __half2*>(&dk[cc / 2]);
+            hm[(cc / 2) & 3] = __hmax2_nan(hm[(cc / 2) & 3], __habs2(hv));
           }
-          pk[c / 2] = pack_half2_rn(p2[0], p2[1]);
-          dk[c / 2] = pack_half2_rn(d2[0], d2[1]);
-          const __half2 h = *reinterpret_cast<const __half2*>(&dk[c / 2]);
-          hm[(c / 2) & 3] = __hmax2_nan(hm[(c / 2) & 3], __habs2(h));
         }
         const __half2 h01 = __hmax2_nan(hm[0], hm[1]), h23 = __hmax2_nan(hm[2], hm[3]);
         const float2 mf = __half22float2(__hmax2_nan(h01, h23));
@@ -367,15 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
-                 const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride, const LhDims& dm,
-                 cudaStream_t st) {
+int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const float* stats, const float* dinv,
+                 float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride, const LhDims& dm, cudaStream_t st) {
   if (kv.q_off % kKTile != 0 || (kv.blocks > 1 && dm.S % kKTile != 0)) return LH_ERR_UNSUPPORTED;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, mst;
   if (make_tmap_f16_3d(&mq, qg, D, dm.S, dm.BH, kQTile) ||
       make_tmap_f16_4d(&mk, kv.k, D, dm.S, dm.BH, kv.blocks, kv.block_stride, kKTile) ||
       make_tmap_f16_4d(&mv, kv.v, D, dm.S, dm.BH, kv.blocks, kv.block_stride, kKTile) ||
-      make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH, kQTile) || make_tmap_f32_3d(&mdq, dqacc, D, dm.S, dm.BH, 32, kQTile))
+      make_tmap_f16_3d(&mdo, dog16, D, dm.S, dm.BH, kQTile) ||
+      make_tmap_f32_3d(&mdq, dqacc, D, dm.S, dm.BH, 32, kQTile) || make_tmap_stats(&mst, stats, dm.S, dm.BH, kQTile))
     return LH_ERR_CUDA;
   const int smem = BwdLayout<D>::BYTES + 1024;
   if (cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -383,7 +372,7 @@ int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const fl
   const int tpb = (dm.S + kKTile - 1) / kKTile;            // key tiles per block
   const int nt = (kv.q_off + dm.S + kKTile - 1) / kKTile;  // key tiles the local queries see
   KernelTimer timer("attn_bwd", st);
-  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, dvec, dinv, dkg, dvg,
+  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mst, dinv, dkg, dvg,
                                                                dkv_block_stride, dm.S, kv.q_off, tpb,
                                                                1.0f / sqrtf((float)D), dm.status);
   return check_launch();
@@ -391,11 +380,10 @@ int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const fl
 
 }  // namespace
 
-int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
-                    const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride,
-                    const LhDims& dm, cudaStream_t st) {
-  return dm.d == 64 ? launch_bwd_t<64>(qg, kv, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st)
-                    : launch_bwd_t<128>(qg, kv, dog16, lse, dvec, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st);
+int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* stats, const float* dinv,
+                    float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride, const LhDims& dm, cudaStream_t st) {
+  return dm.d == 64 ? launch_bwd_t<64>(qg, kv, dog16, stats, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st)
+                    : launch_bwd_t<128>(qg, kv, dog16, stats, dinv, dqacc, dkg, dvg, dkv_block_stride, dm, st);
 }
 
 }  // namespace lh

@@ -49,9 +49,14 @@ int launch_scatter_bwd(const void* dout, const int32_t* idx_g, float* dog, unsig
                        cudaStream_t st);
 // Per-head maximum magnitude of an fp32 [BH, S, d] tensor (amax must start at 0).
 int launch_absmax(const float* x, unsigned int* amax, const LhDims& dm, cudaStream_t st);
-// dog16 = fp16(dog * scale_bh), dvec = <dog16, og>, dinv[bh] = 1/scale_bh, dqacc = 0.
-int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax, void* dog16, float* dvec, float* dinv,
-                    float* dqacc, const LhDims& dm, cudaStream_t st);
+// Rows per head of the attention backward's statistics planes (S rounded up to a multiple of 4, so that each row of
+// the planes starts on a 16-byte boundary for the tensor map).
+__host__ __device__ inline int stats_stride(const LhDims& dm) { return (dm.S + 3) & ~3; }
+// dog16 = fp16(dog * scale_bh), dinv[bh] = 1/scale_bh, dqacc = 0, and the statistics the attention backward reads,
+// stats fp32 [2][BH][stats_stride]: plane 0 = -LSE log2(e) (lse: natural-log LSE of the forward), plane 1 =
+// -<dog16, og> / sqrt(d).
+int launch_bwd_prep(const float* dog, const float* og, const float* lse, const unsigned int* amax, void* dog16,
+                    float* stats, float* dinv, float* dqacc, const LhDims& dm, cudaStream_t st);
 int launch_unpool_bwd(const float* dqg, const float* dkg, const float* dvg, const int32_t* slot, void* dq, void* dk,
                       void* dv, const LhDims& dm, cudaStream_t st);
 // Keys and values of the attention: `blocks` blocks of dm.S rows each (one per rank of a context-parallel group;
@@ -68,12 +73,12 @@ struct KvSource {
 inline KvSource kv_plain(const void* k, const void* v) { return KvSource{k, v, 1, 0, 0}; }
 
 int launch_attn_fwd(const void* qg, const KvSource& kv, float* og, float* lse, const LhDims& dm, cudaStream_t st);
-// qg, dog16: fp16 [BH, S, d] (dog16 scaled per head); dvec scaled alike; dinv: inverse scales.  dqacc (fp32,
-// zeroed) accumulates dQ_g of the local queries; dK_g and dV_g (fp32) of the key rows of block g are written to
-// dkg / dvg + g * dkv_block_stride floats, [BH, S, d] each.
-int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* lse, const float* dvec,
-                    const float* dinv, float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride,
-                    const LhDims& dm, cudaStream_t st);
+// qg, dog16: fp16 [BH, S, d] (dog16 scaled per head); stats from launch_bwd_prep; dinv: inverse scales.  dqacc
+// (fp32, zeroed) accumulates dQ_g of the local queries; dK_g and dV_g (fp32) of the key rows of block g are written
+// to dkg / dvg + g * dkv_block_stride floats, [BH, S, d] each.
+int launch_attn_bwd(const void* qg, const KvSource& kv, const void* dog16, const float* stats, const float* dinv,
+                    float* dqacc, float* dkg, float* dvg, uint64_t dkv_block_stride, const LhDims& dm,
+                    cudaStream_t st);
 
 // Context parallelism: halo rows exchanged between neighbouring ranks (fp32 [BH][L][d], see cp.cu).
 int launch_halo_fwd(const float* og, const int32_t* slot, float* halo, const LhDims& dm, cudaStream_t st);
@@ -89,6 +94,9 @@ int make_tmap_f16_3d(CUtensorMap* map, const void* base, int d, int rows, int bh
 // and 128-byte swizzle.
 int make_tmap_f16_4d(CUtensorMap* map, const void* base, int d, int rows, int bh, int blocks, uint64_t block_stride,
                      int box_rows = 128);
+// Encode the tensor map of the statistics planes of launch_bwd_prep: [2][BH][S] fp32 (row stride stats_stride), box
+// {box_rows, 1, 2} (one sub-tile's rows of both planes), no swizzle; rows beyond S read as zero.
+int make_tmap_stats(CUtensorMap* map, const float* stats, int S, int bh, int box_rows);
 // Encode a 3-D fp32 tensor map over [BH][rows][d] with a {box_cols, box_rows, 1} box, no swizzle.
 int make_tmap_f32_3d(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_cols, int box_rows);
 

@@ -421,10 +421,12 @@ __global__ void __launch_bounds__(256) absmax_kernel(const float* __restrict__ x
 // scale of each head.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__ dog, const float* __restrict__ og,
+                                                       const float* __restrict__ lse,
                                                        const unsigned int* __restrict__ amax, __half* __restrict__ dog16,
-                                                       float* __restrict__ dvec, float* __restrict__ dinv,
+                                                       float* __restrict__ stats, float* __restrict__ dinv,
                                                        float* __restrict__ dqacc, LhDims dm) {
   constexpr int G = D / 8;
+  constexpr float kLog2e = 1.4426950408889634f;
   const int lane = threadIdx.x % G;
   const int64_t total = (int64_t)dm.BH * dm.S;
   const int64_t row0 = (int64_t)blockIdx.x * (256 / G) + threadIdx.x / G;
@@ -449,7 +451,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__
   for (int off = 1; off < G; off <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   if (active) {
     st16(dog16 + row * D + lane * 8, make_uint4(h[0], h[1], h[2], h[3]));
-    if (lane == 0) dvec[row] = dot;
+    if (lane == 0) {
+      const int64_t srow = (int64_t)bh * stats_stride(dm) + row % dm.S;
+      stats[srow] = -lse[row] * kLog2e;
+      stats[(int64_t)dm.BH * stats_stride(dm) + srow] = -dot * rsqrtf((float)D);
+    }
     if (lane == 0 && row % dm.S == 0) dinv[bh] = 1.f / sc;
     const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     store8f(dqacc + row * D + lane * 8, z);
@@ -525,14 +531,16 @@ int launch_absmax(const float* x, unsigned int* amax, const LhDims& dm, cudaStre
   return check_launch();
 }
 
-int launch_bwd_prep(const float* dog, const float* og, const unsigned int* amax, void* dog16, float* dvec, float* dinv,
-                    float* dqacc, const LhDims& dm, cudaStream_t st) {
+int launch_bwd_prep(const float* dog, const float* og, const float* lse, const unsigned int* amax, void* dog16,
+                    float* stats, float* dinv, float* dqacc, const LhDims& dm, cudaStream_t st) {
   const int64_t rows = (int64_t)dm.BH * dm.S;
   KernelTimer timer("bwd_prep", st);
   if (dm.d == 64)
-    bwd_prep_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(dog, og, amax, (__half*)dog16, dvec, dinv, dqacc, dm);
+    bwd_prep_kernel<64><<<blocks_for<64>(rows), 256, 0, st>>>(dog, og, lse, amax, (__half*)dog16, stats, dinv, dqacc,
+                                                              dm);
   else
-    bwd_prep_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(dog, og, amax, (__half*)dog16, dvec, dinv, dqacc, dm);
+    bwd_prep_kernel<128><<<blocks_for<128>(rows), 256, 0, st>>>(dog, og, lse, amax, (__half*)dog16, stats, dinv,
+                                                                dqacc, dm);
   return check_launch();
 }
 
