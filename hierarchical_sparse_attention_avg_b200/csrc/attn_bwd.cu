@@ -6,31 +6,29 @@
 // of its own.
 //
 // One CTA per (head, 128-row key tile); K_j and V_j stay in shared memory while the 64-row query sub-tiles i that
-// can see them (64 i + 63 >= 128 j) stream through.  Warp roles:
-//   warp 0     TMA producer: K_j, V_j once; Q_i and dO_i into a two-stage ring;
-//   warp 1     MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into one of two TMEM buffer pairs,
-//              then, for the previous sub-tile, dV += P^T dO, dK += dS^T Q (accumulated in TMEM for the whole
-//              loop) and dQ^T = K_j^T dS^T (into the consumed S^T columns);
-//   warps 2-5  compute: one key row (TMEM lane) per thread writes the P^T and dS^T rows (fp16) of the sub-tile
-//              to tensor memory, over the S^T and dP^T columns they came from (there they are the A operands of
-//              dV += P^T dO and dK += dS^T Q), and dS^T also to shared memory (the B operand of dQ^T);
-//   warps 6-9  drain: one feature (TMEM lane) per thread moves dQ^T out of TMEM into a shared-memory tile that
-//              one thread adds to the fp32 dQ accumulator with TMA bulk tensor reduce-add.
+// can see them stream through.  Warp roles:
+//   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i and the sub-tile's statistics into a three-stage ring;
+//   warp 1      MMA issuer (one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into one of two TMEM buffer pairs,
+//               then, for the previous sub-tile, dV += P^T dO, dK += dS^T Q (accumulated in TMEM for the whole
+//               loop) and dQ^T = K_j^T dS^T (into the consumed S^T columns);
+//   warps 2-9   compute, two warps per TMEM lane quarter (one key row per thread), each on 32 of the sub-tile's 64
+//               query columns: the P^T and dS^T values (fp16) go to tensor memory over the S^T and dP^T columns
+//               they came from (there they are the A operands of dV += P^T dO and dK += dS^T Q), and dS^T also to
+//               shared memory (the B operand of dQ^T);
+//   warps 10-13 drain: one feature (TMEM lane) per thread moves dQ^T out of TMEM into a shared-memory tile that
+//               one thread adds to the fp32 dQ accumulator with TMA bulk tensor reduce-add.
 // The MMA thread issues S^T/dP^T of sub-tile i+1 before the products of sub-tile i, so the tensor core works while
 // the compute warps do.  64-row sub-tiles keep the double-buffered S^T/dP^T (4 x 64 columns) and the dV/dK
-// accumulators (2 x d columns) inside the 512 tensor-memory columns.
-// Operands are fp16 (gathered Q, K, V exactly; P in [0, 1]; dO_g and dS scaled per head by a power of two so
-// their largest magnitudes sit near 2^10): the layer's window-summed dO_g makes dS and dV sums cancel strongly,
-// and bf16 operands were measured to exceed the 2e-2 + 2e-2|ref| tolerance where fp16 stays within it.  Results
-// are multiplied by the inverse scale; a dS beyond the fp16 range records LH_ERR_RANGE.  For d = 64 the dQ^T
-// product still uses M = 128 (lanes 64..127 ignored).  Every wait is bounded.
+// accumulators (2 x d columns) inside the 512 tensor-memory columns.  Per sub-tile the shared memory carries about
+// 290 KB (operands of the three products with both operands there, TMA writes, dS^T, the dQ staging), which bounds
+// the tensor side at 128 B/clk.
 #include "internal.h"
 
 namespace lh {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kKTile = 128;  // key rows per CTA
 constexpr int kQTile = 64;   // query rows per sub-tile
 constexpr int kStages = 3;   // Q/dO ring depth
@@ -94,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(Lay::B_SF + b), 1);
-      mbar_init(bar(Lay::B_DSF + b), 128);
+      mbar_init(bar(Lay::B_DSF + b), 256);
       mbar_init(bar(Lay::B_MM + b), 1);
       mbar_init(bar(Lay::B_DQF + b), 128);
     }
@@ -163,8 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kQTile / 16; ++kk) {  // reduction over the 64 queries
           const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tDV, tP + kk * 8, sdesc_sw128(sDO + kk * 2048, 8192, 1024), idesc_acc, acc);
-          umma_ts(tDK, tDS + kk * 8, sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc, acc);
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;  // column half h = kk/2 packed at 32 h
+          umma_ts(tDV, tP + pc, sdesc_sw128(sDO + kk * 2048, 8192, 1024), idesc_acc, acc);
+          umma_ts(tDK, tDS + pc, sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc, acc);
         }
 #pragma unroll
         for (int kk = 0; kk < kKTile / 16; ++kk)  // reduction over the 128 keys
@@ -198,9 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(bar(Lay::B_DRAIN));
       mbar_wait_teardown(bar(Lay::B_DRAIN), 0);
     }
-  } else if (warp < 6) {
-    // ---------------------------------------------------------------- compute: P^T and dS^T rows
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- compute: P^T and dS^T, one key row per
+    // thread, 32 query columns (half hc of the sub-tile) per warp
     const int quarter = warp & 3;
+    const int hc = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;  // key row inside the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int key = kt * kKTile + r;  // global key row
@@ -209,38 +210,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < nit && ok; ++it) {
       const int b = it & 1, s = it % kStages, i = i0 + it;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_SF + b), (it >> 1) & 1, &s_wait, status));
-      // the sub-tile's statistics arrived with its Q/dO stage (complete before S^T was issued)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QF + s), (it / kStages) & 1, &s_wait, status));
       if (!ok) break;
-      float sv[64], dp[64];
+      float sv[32], dp[32];
       tc_fence_after();
-      tmem_ld32(tmem + 128 * b + lane_base, *reinterpret_cast<float(*)[32]>(&sv[0]));
-      tmem_ld32(tmem + 128 * b + lane_base + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
-      tmem_ld32(tmem + 128 * b + 64 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[0]));
-      tmem_ld32(tmem + 128 * b + 96 + lane_base, *reinterpret_cast<float(*)[32]>(&dp[32]));
+      tmem_ld32(tmem + 128 * b + lane_base + 32 * hc, sv);
+      tmem_ld32(tmem + 128 * b + 64 + lane_base + 32 * hc, dp);
       tmem_ld_wait();
-      uint32_t pk[32], dk[32];
+      uint32_t pk[16], dk[16];
       {
-        const int qg0 = q_off + i * kQTile;  // global row of the sub-tile's first query
-        const bool diag = qg0 < key;         // some query of the sub-tile precedes the key (masked)
-        // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D) scale = P fma(dP, scale, -D scale), two columns per
-        // packed fp32x2 instruction; the statistics are stored negated, as 16-byte broadcast vectors.  The fp16
-        // range of dS is checked on the packed values (beyond it: an infinity; NaN stays NaN): largest |dS| half2
-        // over 4 independent chains
+        const int qg0 = q_off + i * kQTile + 32 * hc;  // global row of this half's first query
+        const bool diag = qg0 < key;
         __half2 hm[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) hm[k] = __float2half2_rn(0.f);
-        const ulonglong2* nl4 = reinterpret_cast<const ulonglong2*>(smem + Lay::STAT + s * Lay::ST);
-        const ulonglong2* nd4 = nl4 + kQTile / 4;
+        const ulonglong2* nl4 = reinterpret_cast<const ulonglong2*>(smem + Lay::STAT + s * Lay::ST) + 8 * hc;
+        const ulonglong2* nd4 = reinterpret_cast<const ulonglong2*>(smem + Lay::STAT + s * Lay::ST + kQTile * 4) + 8 * hc;
 #pragma unroll
-        for (int c = 0; c < kQTile; c += 4) {
+        for (int c = 0; c < 32; c += 4) {
           const ulonglong2 nl = nl4[c >> 2], nd = nd4[c >> 2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int cc = c + 2 * h;
             const uint64_t arg = fma_f32x2(f2pack(sv[cc], sv[cc + 1]), scl2, h ? nl.y : nl.x);
             float p0 = ex2(f2lo(arg)), p1 = ex2(f2hi(arg));
-            if (diag) {  // queries that precede the key do not see it
+            if (diag) {
               if (qg0 + cc < key) p0 = 0.f;
               if (qg0 + cc + 1 < key) p1 = 0.f;
             }
@@ -256,24 +250,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 mf = __half22float2(__hmax2_nan(h01, h23));
         if (__any_sync(0xffffffffu, !(mf.x <= 65504.f && mf.y <= 65504.f)) && lane == 0)
           set_status(status, LH_ERR_RANGE);
-        // P/dS buffer b is free once the products of sub-tile it-2 have completed
         if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_MM + b), ((it >> 1) - 1) & 1, &s_wait,
                                                             status));
       }
       if (ok) {
-        // P^T and dS^T rows to tensor memory (A operands of dV and dK), dS^T also to shared memory (B of dQ^T)
-        float pf[32], df[32];
-#pragma unroll
-        for (int w = 0; w < 32; ++w) {
-          pf[w] = __uint_as_float(pk[w]);
-          df[w] = __uint_as_float(dk[w]);
-        }
-        tmem_st32(tmem + 128 * b + lane_base, pf);
-        tmem_st32(tmem + 128 * b + 64 + lane_base, df);
+        tmem_st16(tmem + 128 * b + lane_base + 32 * hc, pk);
+        tmem_st16(tmem + 128 * b + 64 + lane_base + 32 * hc, dk);
         uint8_t* sDS = smem + Lay::DS + b * Lay::PT;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunk ch holds queries 8 ch .. 8 ch + 7
-          const uint32_t off = sw128_offset(r, ch);
+        for (int ch = 0; ch < 4; ++ch) {  // 16-byte chunk 4 hc + ch holds queries 8 (4 hc + ch) .. + 7
+          const uint32_t off = sw128_offset(r, 4 * hc + ch);
           *reinterpret_cast<uint4*>(sDS + off) = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
         }
         fence_proxy_async_smem();
@@ -282,28 +268,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(Lay::B_DSF + b));
       }
     }
-    // epilogue: dV and dK rows of this key tile (the products' accumulators are final after B_FIN)
-    ok = named_barrier_and(kBarCompute, 128, ok);
+    // epilogue: dV (column half 0's warps) or dK (half 1's) rows of this key tile, final after B_FIN
+    ok = named_barrier_and(kBarCompute, 256, ok);
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FIN), 0, &s_wait, status));
     if (ok) {
       tc_fence_after();
+      const uint32_t tacc = hc == 0 ? tDV : tDK;
+      float* dst_base = hc == 0 ? dvg : dkg;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tacc = which == 0 ? tDV : tDK;
-        float* dst_base = which == 0 ? dvg : dkg;
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        tmem_ld32(tacc + lane_base + c * 32, v);
+        tmem_ld_wait();
+        if (krow0 + r < S) {
+          float4* dst = reinterpret_cast<float4*>(dst_base + kblk * dkv_block_stride +
+                                                  ((int64_t)bh * S + krow0 + r) * D + c * 32);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(tacc + lane_base + c * 32, v);
-          tmem_ld_wait();
-          if (krow0 + r < S) {  // the key row exists (the last tile of a single ragged block is partial)
-            float4* dst = reinterpret_cast<float4*>(dst_base + kblk * dkv_block_stride +
-                                                    ((int64_t)bh * S + krow0 + r) * D + c * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
-                                    v[q4 * 4 + 3] * inv_scale);
-          }
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_float4(v[q4 * 4 + 0] * inv_scale, v[q4 * 4 + 1] * inv_scale, v[q4 * 4 + 2] * inv_scale,
+                                  v[q4 * 4 + 3] * inv_scale);
         }
       }
     }
@@ -311,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- drain: dQ^T -> shared tile -> TMA reduce-add
     const int quarter = warp & 3;
     const int f = quarter * 32 + lane;  // feature = TMEM lane of dQ^T
-    const int dt = threadIdx.x - 192;   // 0..127 inside the drain group
+    const int dt = threadIdx.x - 320;   // 0..127 inside the drain group
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     float* stage = reinterpret_cast<float*>(smem + Lay::DQ);
     bool ok = true;
