@@ -34,6 +34,8 @@ constexpr int kQTile = 64;   // query rows per sub-tile
 constexpr int kStages = 3;   // Q/dO ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBarCompute = 1, kBarDrain = 2;  // named barrier ids (0 is __syncthreads)
+// Below this many key tiles per head the grid runs head-fastest (one head's CTAs do not fill the 148 SMs).
+constexpr int kHeadFastBelow = 148;
 
 template <int D>
 struct BwdLayout {
@@ -61,8 +63,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmST,
                     const float* __restrict__ dinv, float* __restrict__ dkg,
-                    float* __restrict__ dvg, uint64_t dkv_block_stride, int S, int q_off, int kv_tpb, float scale,
-                    int* status) {
+                    float* __restrict__ dvg, uint64_t dkv_block_stride, int S, int q_off, int kv_tpb, int head_fast,
+                    float scale, int* status) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
@@ -74,8 +76,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // key tiles are numbered globally (tile kt is tile kt % kv_tpb of block kt / kv_tpb); the S local query rows are
   // global rows q_off .. q_off + S - 1 (q_off = 0 without context parallelism, else a multiple of 128)
-  const int kt = blockIdx.x;  // key tile: tile 0 meets the most query sub-tiles and is scheduled first
-  const int bh = blockIdx.y;
+  // key tile: tile 0 meets the most query sub-tiles and is scheduled first; with head_fast the head is the grid's
+  // fastest index (short sequences: every head's heavy tiles start in the first wave)
+  const int kt = head_fast ? blockIdx.y : blockIdx.x;
+  const int bh = head_fast ? blockIdx.x : blockIdx.y;
   const int kblk = kt / kv_tpb, krow0 = (kt % kv_tpb) * kKTile;  // block of the key tile and its first row there
   const int nq = (S + kQTile - 1) / kQTile;
   const int i0 = max(0, 2 * kt - q_off / kQTile);  // first local sub-tile with a query at or after the tile's first key
@@ -355,9 +359,10 @@ int launch_bwd_t(const void* qg, const KvSource& kv, const void* dog16, const fl
   const int tpb = (dm.S + kKTile - 1) / kKTile;            // key tiles per block
   const int nt = (kv.q_off + dm.S + kKTile - 1) / kKTile;  // key tiles the local queries see
   KernelTimer timer("attn_bwd", st);
-  attn_bwd_kernel<D><<<dim3(nt, dm.BH), kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mst, dinv, dkg, dvg,
-                                                               dkv_block_stride, dm.S, kv.q_off, tpb,
-                                                               1.0f / sqrtf((float)D), dm.status);
+  const int head_fast = nt < kHeadFastBelow;
+  const dim3 grid = head_fast ? dim3(dm.BH, nt) : dim3(nt, dm.BH);
+  attn_bwd_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mst, dinv, dkg, dvg, dkv_block_stride, dm.S,
+                                                   kv.q_off, tpb, head_fast, 1.0f / sqrtf((float)D), dm.status);
   return check_launch();
 }
 
