@@ -347,6 +347,81 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_cp(args, w):
+    """Context-parallel step: rank r holds tokens [r N/G, (r+1) N/G) of every head of one sequence and runs the
+    lh_cp_* stages with NCCL all-gathers and a reduce-scatter (cp.forward / cp.backward); the step time is the max
+    over ranks and the tokens are the one sequence's (strong scaling).  A single process forms a group of one."""
+    import datetime
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world == 1:  # a group of one: under torchrun its rendezvous variables are set, else a local port is taken
+        if "MASTER_ADDR" not in os.environ:
+            import socket
+
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0", WORLD_SIZE="1")
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    from hierarchical_sparse_attention_avg_b200 import cp, lh
+    from hierarchical_sparse_attention_avg_b200.inputs import make_inputs
+
+    P = lh.Params(**w)
+    sp = cp.split(P, world)
+    L = sp.local
+    q, k, v, dout = make_inputs(L.B, L.H, L.N, L.d, seed=rank, device=dev)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    st = cp.new_state(sp, rank, dev)
+    ex = cp.TorchDistExchange()
+
+    def step():
+        cp.forward(st, q, k, v, ex, o=o)
+        cp.backward(st, dout, ex, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    torch.distributed.barrier()
+    clocks = make_clock_sampler(dev)
+    clocks.start()
+    lh.lh_profile_enable(True)
+    lh.lh_profile_read()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    torch.distributed.barrier()
+    lh.lh_profile_enable(False)
+    prof = lh.lh_profile_read()
+    clk = clocks.stop()
+    t = torch.tensor([e0.elapsed_time(e1) / args.steps, float(lh.lh_get_status(dev))], dtype=torch.float64,
+                     device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms, status = float(t[0]), int(t[1])
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {lh.error_string(status)}")
+    if rank == 0:
+        tokens = w["B"] * w["N"]
+        kernels = {n: {"launches": c, "ms": m / c} for n, (c, m) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+        line = {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, **w, "S": kernel_work(w)[1], "S_per_rank": sp.S_local,
+                           "parallelism": f"cp{world}",
+                           "exchange_bytes_per_rank": {"kv_all_gather": sp.kv_bytes * world,
+                                                       "halo_all_gathers": 2 * sp.halo_bytes * world,
+                                                       "dkv_reduce_scatter": sp.dkv_bytes * world}},
+                "kernels": kernels, "gpu_launches": sum(c for c, _ in prof.values()), "clocks": clk, "e2e": None}
+        print(json.dumps(line), flush=True)
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -356,10 +431,16 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallelism: the ranks split ONE sequence of the workload (strong scaling), "
+                         "exchanging through lh_cp_* and NCCL collectives; default: independent replicas")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.cp:
+        run_cp(args, w)
         return
 
     world, rank, local = dist_setup()
