@@ -93,7 +93,7 @@ __device__ __forceinline__ bool zero_or_normal(float x) {
 // kScore: 0 = no scores; 1 = score levels 0..L-2; 2 = score levels 1..L-1 (children-expansion variant).  Scored
 // level l is written at row dm.soff[l] of the head's score array.
 template <int D, int P, int L, int kScore>
-__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, LhDims dm) {
+__device__ __forceinline__ void pool_score_body(const PoolJob& job, unsigned block, const LhDims& dm) {
   constexpr int G = D / 8;
   constexpr int GPB = kPoolThreads / G;
   constexpr int W = ipow(P, L - 1);
@@ -102,9 +102,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
   static_assert(TB % P == 0, "batch must hold whole level-1 entries");
   extern __shared__ uint4 s_raw[];    // [kPoolStages][TB][kPoolThreads]
 
-  const PoolJob& job = jobs.job[blockIdx.y];
   const int lane = threadIdx.x % G;
-  const int64_t group = (int64_t)blockIdx.x * GPB + threadIdx.x / G;
+  const int64_t group = (int64_t)block * GPB + threadIdx.x / G;
   const int nblk = dm.N / W;
   const int64_t total = (int64_t)dm.BH * nblk;
   const bool active = group < total;
@@ -234,6 +233,19 @@ __global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs,
       }
     }
   }
+}
+
+// One launch for every job; the job is the grid's fastest index, so each SM holds blocks of every job at once: the
+// scored job's blocks are bound by instruction issue, the others by memory, and they overlap.  kScore is the scored
+// job's mode (jobs without a score array run the unscored body).
+template <int D, int P, int L, int kScore>
+__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, int njobs, LhDims dm) {
+  const int ji = (int)(blockIdx.x % (unsigned)njobs);
+  const unsigned block = blockIdx.x / (unsigned)njobs;
+  if (kScore != 0 && jobs.job[ji].scores != nullptr)
+    pool_score_body<D, P, L, kScore>(jobs.job[ji], block, dm);
+  else
+    pool_score_body<D, P, L, 0>(jobs.job[ji], block, dm);
 }
 
 // ---- Gather (step 4).  One warp per gathered row: lane i holds features [2*NW*i, 2*NW*i + 2*NW) (NW 32-bit
@@ -506,32 +518,27 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherJobs jo
   if (overflow) set_status(dm.status, LH_ERR_RANGE);
 }
 
-// Jobs with scores and jobs without run as two launches of the two specialisations (the one without carries no
-// scoring code and fewer registers).
 template <int D, int P, int L, int kScore>
-int launch_pool_kind(const PoolJobs& all, int njobs, const LhDims& dm, cudaStream_t st) {
-  PoolJobs jobs;
-  int n = 0;
-  for (int i = 0; i < njobs; ++i)
-    if ((all.job[i].scores != nullptr) == (kScore != 0)) jobs.job[n++] = all.job[i];
-  if (n == 0) return LH_OK;
+int launch_pool_kind(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
   constexpr int G = D / 8;
   constexpr int W = ipow(P, L - 1);
   const int64_t groups = (int64_t)dm.BH * (dm.N / W);
   const int64_t blocks = (groups + kPoolThreads / G - 1) / (kPoolThreads / G);
-  if (blocks > 0x7fffffff) return LH_ERR_UNSUPPORTED;
+  if (blocks * njobs > 0x7fffffff) return LH_ERR_UNSUPPORTED;
   const int smem = kPoolStages * pool_batch(W) * kPoolThreads * (int)sizeof(uint4);
   auto kernel = pool_score_kernel<D, P, L, kScore>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LH_ERR_CUDA;
-  kernel<<<dim3((unsigned)blocks, n), kPoolThreads, smem, st>>>(jobs, dm);
+  kernel<<<(unsigned)(blocks * njobs), kPoolThreads, smem, st>>>(jobs, njobs, dm);
   return check_launch();
 }
 
 template <int D, int P, int L>
 int launch_pool_t(const PoolJobs& jobs, int njobs, const LhDims& dm, cudaStream_t st) {
-  const int rc = launch_pool_kind<D, P, L, 0>(jobs, njobs, dm, st);
-  if (rc != LH_OK) return rc;
+  if (njobs <= 0) return LH_OK;
+  bool scored = false;
+  for (int i = 0; i < njobs; ++i) scored |= jobs.job[i].scores != nullptr;
+  if (!scored) return launch_pool_kind<D, P, L, 0>(jobs, njobs, dm, st);
   return dm.expand ? launch_pool_kind<D, P, L, 2>(jobs, njobs, dm, st) : launch_pool_kind<D, P, L, 1>(jobs, njobs, dm, st);
 }
 
