@@ -5,8 +5,10 @@
 // attention and scatter all work within one head), so the step runs in chunks of consecutive heads of one batch
 // row: chunk g's host-to-device copies (on the caller's h2d stream), its lh_forward + lh_backward (on the compute
 // stream) and its device-to-host copies (on the d2h stream) overlap with the neighbouring chunks', and the two copy
-// directions share the full-duplex link.  Two chunks' tensors are resident at a time (slots 0 and 1 of the
-// caller's device buffer); one context and one workspace serve every chunk, in order, on the compute stream.
+// directions share the full-duplex link.  Three chunks' tensors are resident at a time (slots 0..2 of the caller's
+// device buffer): chunk g's inputs are copied in while chunk g-1 is computed and chunk g-2 is copied out, so
+// neither copy direction waits for a computation; one context and one workspace serve every chunk, in order, on
+// the compute stream.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,7 +18,7 @@
 
 namespace {
 
-constexpr int kSlots = 2;
+constexpr int kSlots = 3;
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -70,13 +72,14 @@ int events_for_current_device(StepEvents** out) {
   StepEvents& e = g_events[dev];
   if (!e.ready) {
     // create all events or none: on a failure the ones already created are destroyed
-    cudaEvent_t* all[1 + 3 * kSlots] = {&e.start};
+    constexpr int kPer = 3;  // events per slot
+    cudaEvent_t* all[1 + kPer * kSlots] = {&e.start};
     for (int s = 0; s < kSlots; ++s) {
-      all[1 + 3 * s] = &e.h2d[s];
-      all[2 + 3 * s] = &e.comp[s];
-      all[3 + 3 * s] = &e.d2h[s];
+      all[1 + kPer * s] = &e.h2d[s];
+      all[2 + kPer * s] = &e.comp[s];
+      all[3 + kPer * s] = &e.d2h[s];
     }
-    for (int i = 0; i < 1 + 3 * kSlots; ++i) {
+    for (int i = 0; i < 1 + kPer * kSlots; ++i) {
       if (cudaEventCreateWithFlags(all[i], cudaEventDisableTiming) != cudaSuccess) {
         for (int j = 0; j < i; ++j) cudaEventDestroy(*all[j]);
         return LH_ERR_CUDA;

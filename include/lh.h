@@ -236,7 +236,7 @@ int lh_score_topk_static(const lh_params* P, const void* k, const float* scores_
 /* ---- host-resident step ------------------------------------------------------------------------------ */
 
 /* Device bytes lh_step_host needs with chunks of `heads_per_chunk` heads (0 if P is invalid or heads_per_chunk
- * does not divide H): two chunks' eight tensors, one chunk's ctx and one chunk's workspace. */
+ * does not divide H): three chunks' eight tensors, one chunk's ctx and one chunk's workspace. */
 size_t lh_step_host_bytes(const lh_params* P, int heads_per_chunk);
 
 /* The pages have no counterpart to this entry point: it serves callers whose tensors live in host memory.

@@ -127,7 +127,7 @@ def test_step_host_bytes_and_argument_errors(lh):
     tensor = 2 * 4096 * 64 * 2  # one chunk tensor of two heads, bf16
     need = lh.lh_step_host_bytes(P, 2)
     rnd = lambda x: (x + 255) // 256 * 256
-    assert need == 2 * 8 * rnd(tensor) + rnd(lh.lh_ctx_bytes(Pc)) + rnd(lh.lh_workspace_bytes(Pc))
+    assert need == 3 * 8 * rnd(tensor) + rnd(lh.lh_ctx_bytes(Pc)) + rnd(lh.lh_workspace_bytes(Pc))
     assert lh.lh_step_host_bytes(P, 3) == 0  # does not divide H
     assert lh.lh_step_host_bytes(P, 0) == 0
     bad = lh.Params(1, 2, 4100, 64, 3, 4, 256, 8)  # p^(L-1) = 16 does not divide N
