@@ -231,17 +231,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i)
               if (c * 32 + i > row) s[c][i] = -INFINITY;
         }
-        // row max of the raw scores (the scale is positive), as 8 independent chains
+        // row max of the raw scores (the scale is positive), as 8 independent chains: chain k takes columns
+        // k, k + 8, ..., k + 120, two new ones per three-input max
+        auto col = [&](int x) { return s[x >> 5][x & 31]; };
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(s[0][k], s[0][k + 8]);
+        for (int k = 0; k < 8; ++k) {
+          float m = fmax3(col(k), col(k + 8), col(k + 16));
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c > 0 || i >= 16) mx8[i & 7] = fmaxf(mx8[i & 7], s[c][i]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+          for (int t = 3; t + 1 < 16; t += 2) m = fmax3(m, col(k + 8 * t), col(k + 8 * t + 8));
+          mx8[k] = fmaxf(m, col(k + 120));
+        }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) *
                          scale_log2;
         // The reference max moves only when some row of the warp exceeds it by more than kSlack (log2 units):
         // P = 2^(s scale - m_ref) then stays in [0, 2^kSlack], well inside fp16, and O is rescaled rarely.
@@ -254,8 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = m_new;
         }
         // P = 2^(s * scale - m) in fp16 over the first 64 columns of S (each half stored as soon as it
-        // is packed, so the scores it came from are dead), and its row sum
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // is packed, so the scores it came from are dead), and its row sum; arguments and sums as fp32 pairs
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+        const uint64_t scl2 = f2pack(scale_log2, scale_log2), nm2 = f2pack(-m_run, -m_run), one2 = f2pack(1.f, 1.f);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float pk[32];
@@ -263,13 +265,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 2 * h; c < 2 * h + 2; ++c)
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              const float p0 = ex2(fmaf(s[c][i], scale_log2, -m_run));
-              const float p1 = ex2(fmaf(s[c][i + 1], scale_log2, -m_run));
-              rs8[(i >> 1) & 7] += p0 + p1;
+              const uint64_t arg = fma_f32x2(f2pack(s[c][i], s[c][i + 1]), scl2, nm2);
+              const float p0 = ex2(f2lo(arg)), p1 = ex2(f2hi(arg));
+              const uint64_t p2 = f2pack(p0, p1);
+              rs2[(i >> 1) & 3] = fma_f32x2(p2, one2, rs2[(i >> 1) & 3]);
               pk[(c & 1) * 16 + i / 2] = __uint_as_float(pack_half2_rn(p0, p1));
             }
           tmem_st32(tS + 32 * h, pk);
         }
+        float rs8[8] = {f2lo(rs2[0]), f2hi(rs2[0]), f2lo(rs2[1]), f2hi(rs2[1]),
+                        f2lo(rs2[2]), f2hi(rs2[2]), f2lo(rs2[3]), f2hi(rs2[3])};
         // O_q += P_q,j-1 V_j-1 has completed (it was issued before S_q,j): bring O_q to the new max
         if (j > 0 && move) {
 #pragma unroll
