@@ -347,48 +347,97 @@ __global__ void __launch_bounds__(kWinThreads, 4) window_sum_kernel(const float*
   cp_async_wait<0>();
 }
 
-// Small blocks (many per SM) for the scatter backward: a gathered row sums a window of 1 to p^(L-1) upstream rows,
-// and a block retires only with its slowest row.
-constexpr int kSbThreads = 64;
+// Scatter backward.  A gathered row sums a window of 1 to p^(L-1) upstream rows, so a row group that summed its
+// own row's whole window would keep its block alive for the longest window (eight round trips for a 64-row
+// window) while most rows need one.  Instead the windows of the block's rows (one row per row group) are cut into
+// chunks of up to kSbChunk consecutive upstream rows, numbered row by row; in each round every row group loads and
+// sums one chunk (all its rows in flight at once) into a shared slot, and after the round's barrier each row group
+// adds the slots of its own row in chunk order.  The order of every addition is fixed by the row's window, so the
+// result does not depend on the schedule.
+constexpr int kSbThreads = 256;
+constexpr int kSbChunk = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kSbThreads) scatter_bwd_kernel(const __nv_bfloat16* __restrict__ dout,
                                                                  const int32_t* __restrict__ idx_g,
                                                                  float* __restrict__ dog,
                                                                  unsigned int* __restrict__ amax, LhDims dm) {
-  constexpr int G = D / 8;
-  const int lane = threadIdx.x % G;
+  constexpr int G = D / 8;             // lanes per row
+  constexpr int NG = kSbThreads / G;   // row groups = rows per block (16 or 32)
+  __shared__ int64_t s_src[NG];        // element offset of the row's first upstream row
+  __shared__ int s_len[NG];            // upstream rows in the row's window (0: no row)
+  __shared__ int s_base[NG + 1];       // first chunk of each row; s_base[NG] = chunks of the block
+  __shared__ __align__(16) float s_part[2][NG][D];
+  const int lane = threadIdx.x % G, g = threadIdx.x / G;
   const int64_t total = (int64_t)dm.BH * dm.S;
-  const int64_t row0 = (int64_t)blockIdx.x * (kSbThreads / G) + threadIdx.x / G;
+  const int64_t row0 = (int64_t)blockIdx.x * NG + g;
   const bool active = row0 < total;
   const int64_t row = active ? row0 : total - 1;
   const int bh = (int)(row / dm.S);
-  const int gid = idx_g[row];
-  const int lev = level_of(gid, dm);
-  const int j = gid - dm.off[lev];
-  const int w = dm.wl[lev];
-  const int t0 = (j + 1) * w - 1;
-  const int t1 = min(t0 + w - 1, dm.N - 1);
-  const __nv_bfloat16* src = dout + ((int64_t)bh * dm.N) * D + lane * 8;
+  if (lane == 0) {
+    int len = 0;
+    int64_t src = 0;
+    if (active) {
+      const int gid = idx_g[row];
+      const int lev = level_of(gid, dm);
+      const int j = gid - dm.off[lev];
+      const int w = dm.wl[lev];
+      const int t0 = (j + 1) * w - 1;
+      const int t1 = min(t0 + w - 1, dm.N - 1);
+      len = t1 - t0 + 1;
+      src = ((int64_t)bh * dm.N + t0) * D;
+    }
+    s_len[g] = len;
+    s_src[g] = src;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // chunk counts, inclusive scan over the row groups
+    const int r = threadIdx.x;
+    int c = r < NG ? (s_len[r] + kSbChunk - 1) / kSbChunk : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, c, off);
+      if (r >= off) c += y;
+    }
+    if (r < NG) s_base[r + 1] = c;
+    if (r == 0) s_base[0] = 0;
+  }
+  __syncthreads();
+  const int T = s_base[NG], first = s_base[g], last = s_base[g + 1];
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int t = t0;
-  for (; t + 7 <= t1; t += 8) {  // eight rows in flight
-    uint4 r[8];
+  for (int w0 = 0, b = 0; w0 < T; w0 += NG, b ^= 1) {
+    const int tau = w0 + g;  // this row group's chunk in the round
+    if (tau < T) {
+      int r = 0;  // the row of chunk tau: the last r with s_base[r] <= tau
 #pragma unroll
-    for (int u = 0; u < 8; ++u) r[u] = ld_stream16(src + (int64_t)(t + u) * D);
+      for (int step = NG / 2; step > 0; step >>= 1)
+        if (s_base[r + step] <= tau) r += step;
+      const int c = tau - s_base[r];
+      const int n = min(kSbChunk, s_len[r] - c * kSbChunk);
+      const __nv_bfloat16* src = dout + s_src[r] + (int64_t)c * kSbChunk * D + lane * 8;
+      uint4 v[kSbChunk];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kSbChunk; ++u)
+        if (u < n) v[u] = ld_stream16(src + (int64_t)u * D);
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int u = 0; u < kSbChunk; ++u) {
+        if (u < n) {
+          float f[8];
+          unpack8(v[u], f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part[i] += f[i];
+        }
+      }
+      store8f(&s_part[b][g][lane * 8], part);
+    }
+    __syncthreads();  // the round's slots are written (and the slots of two rounds back were read by their owners)
+    for (int t = max(first, w0); t < min(last, w0 + NG); ++t) {
       float f[8];
-      unpack8(r[u], f);
+      load8f(&s_part[b][t - w0][lane * 8], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += f[i];
     }
-  }
-  for (; t <= t1; ++t) {
-    float f[8];
-    unpack8(ld_stream16(src + (int64_t)t * D), f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += f[i];
   }
   if (active) store8f(dog + row * D + lane * 8, acc);
   if (amax) {
