@@ -313,6 +313,14 @@ def w_name(w):
     return "custom"
 
 
+def arm_config(args, w, world: int) -> dict:
+    """The `config` of the bench line, the same for both arms (the reference arm times a sample of this workload)."""
+    S = kernel_work(w)[1]
+    l2 = ("inputs larger than L2 (2 GB per tensor), no flush" if w["B"] * w["H"] * w["N"] * w["d"] * 2 > 126e6
+          else "inputs smaller than L2, no flush")
+    return {"workload": args.workload, **w, "S": S, "parallelism": f"replicas{world}", "l2": l2}
+
+
 def run_reference(args, w):
     """The oracle as the reference arm: W warm-up steps and K timed steps, each one head of the workload
     (forward + backward) on the host cores; tokens/s of that sample.  Rank 0 only."""
@@ -339,7 +347,7 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w_name(w), **w, "sample": sample},
+            "config": arm_config(args, w, int(os.environ.get("WORLD_SIZE", "1"))),
             "scaled_to_all_heads": {"ms_per_step": sec * 1e3 * heads,
                                     "note": f"one head's time x {heads} heads: the time the whole step would take"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
@@ -557,9 +565,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": args.workload, **w, "S": S, "parallelism": f"replicas{world}",
-                           "l2": "inputs larger than L2 (2 GB per tensor), no flush"
-                           if w["B"] * w["H"] * w["N"] * w["d"] * 2 > 126e6 else "inputs smaller than L2, no flush"},
+                "config": arm_config(args, w, world),
                 "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
                 "clocks": clk, "e2e": e2e}
         if world == 1 and not args.no_cpu_baseline:
