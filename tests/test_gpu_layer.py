@@ -25,6 +25,7 @@ CASES = {
     "whole-pyramid": (1, 2, 1024, 64, 3, 4, 1024, 4),  # k >= every level: S = 1344
     "p2-L5": (1, 1, 2048, 64, 5, 2, 64, 2),
     "p8-L3-B2": (2, 1, 4096, 128, 3, 8, 64, 4),
+    "p8-L4-wide": (1, 1, 8192, 64, 4, 8, 64, 8),     # coarsest windows of 512 rows, S = 208
     # the pages' recipe parameters L=3, p=4, k=1536 ([C] "The Core Innovation"), C=16: 96 picks per chunk, S = 4096
     "recipe-L3-k1536": (1, 1, 16384, 64, 3, 4, 1536, 16),
     # children-expansion variant (LH_EXPAND_CHILDREN): level l keeps the p children of level l+1's picks
