@@ -29,6 +29,11 @@ constexpr int kTile = 128;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSlack = 8.0f;  // largest log2 of P
+// Below this many CTAs (query-tile pairs) per head the grid runs head-fastest, so every head's longest CTAs start
+// in the first waves instead of trailing the grid (512K, S = 20K: 1.67 -> 1.56 ms); above it the pairs of one head
+// run together and share its keys and values in L2, which dominates at very long S (dense 512K: 1024 ms against
+// 1267 head-fastest).
+constexpr int kHeadFastBelow = 512;
 
 template <int D>
 struct FwdLayout {
@@ -47,7 +52,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, float* __restrict__ og, float* __restrict__ lse, int S,
-                    int npair, int q_tile0, int kv_tpb, float scale_log2, int* status) {
+                    int npair, int q_tile0, int kv_tpb, int head_fast, float scale_log2, int* status) {
   using Lay = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
@@ -57,10 +62,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](uint32_t i) { return sb + Lay::BAR + 8u * i; };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // heaviest pairs first, the head being the grid's fastest index: every head's heavy pairs start in the first
-  // waves, so the longest CTAs do not trail the grid (512K: 1.77 -> 1.69 ms against pairs fastest)
-  const int pt = npair - 1 - (int)blockIdx.y;
-  const int bh = blockIdx.x;
+  // heaviest pairs first; with head_fast the head is the grid's fastest index
+  const int pt = npair - 1 - (int)(head_fast ? blockIdx.y : blockIdx.x);
+  const int bh = head_fast ? blockIdx.x : blockIdx.y;
   const int ntile = (S + kTile - 1) / kTile;
   const bool v1 = 2 * pt + 1 < ntile;    // the pair's second query tile exists
   // key tiles are numbered globally: the local query tile t is global tile q_tile0 + t (context parallelism puts
@@ -339,9 +343,9 @@ int launch_fwd_t(const void* qg, const KvSource& kv, float* og, float* lse, cons
   const int npair = (nt + 1) / 2;
   const float scale_log2 = kLog2e / sqrtf((float)D);
   KernelTimer timer("attn_fwd", st);
-  if (npair > 65535) return LH_ERR_UNSUPPORTED;  // the grid's y extent (S above 16.7M gathered rows)
-  const dim3 grid(dm.BH, npair);
-  attn_fwd_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, npair, kv.q_off / kTile, nt,
+  const int head_fast = npair < kHeadFastBelow;
+  const dim3 grid = head_fast ? dim3(dm.BH, npair) : dim3(npair, dm.BH);
+  attn_fwd_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, og, lse, dm.S, npair, kv.q_off / kTile, nt, head_fast,
                                                    scale_log2, dm.status);
   return check_launch();
 }
