@@ -42,6 +42,36 @@ __device__ __forceinline__ float row_score(const double (&x)[8]) {
   return f32_rn_of(s);
 }
 
+// This lane's share of a row's score: the squares of its 8 values summed left to right in fp64.
+__device__ __forceinline__ double lane_sq8(const float (&xf)[8]) {
+  double s = f64_of(xf[0]) * f64_of(xf[0]);
+#pragma unroll
+  for (int i = 1; i < 8; ++i) s = fma(f64_of(xf[i]), f64_of(xf[i]), s);
+  return s;
+}
+
+// Scores of 4 rows at once from each lane's shares part[u] (row u of the group of 4).  The pairwise tree over a
+// row's G lanes is the xor butterfly of row_score (partners L^1, then L^2, ...); its first two rounds are done
+// transposed: in round m each lane keeps half of its remaining rows (the upper half when bit m of the lane is set)
+// and adds its partner's shares of those rows, which the partner sends; the later rounds (L^4, L^8) pair lanes that
+// hold the same row.  Every addition has the same two operands as in the per-row butterfly, so the sums are
+// bit-identical, and lane L ends with the score of row 2 (L & 1) + ((L >> 1) & 1).  Returns that row.
+template <int G>
+__device__ __forceinline__ int rows4_score(const double (&part)[4], int lane, float& score) {
+  const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
+  double r2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const double got = __shfl_xor_sync(0xffffffffu, b0 ? part[i] : part[i + 2], 1);
+    r2[i] = (b0 ? part[i + 2] : part[i]) + got;
+  }
+  double r = (b1 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? r2[0] : r2[1], 2);
+#pragma unroll
+  for (int off = 4; off < G; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+  score = f32_rn_of(r);
+  return 2 * b0 + b1;
+}
+
 // Round 8 fp64 sums / w to bf16 (single rounding), returning packed bits and the bf16 values as fp64.
 __device__ __forceinline__ uint4 round_pooled(const double (&sum)[8], double inv_w, double (&val)[8]) {
   uint32_t b[8];
@@ -138,14 +168,20 @@ __device__ __forceinline__ void pool_score_body(const PoolJob& job, unsigned blo
     const int t0 = bi * TB;
     const uint4* raw_s = my + (bi % kPoolStages) * TB * kPoolThreads;  // row u at raw_s[u * kPoolThreads]
 
+    // level 0 is scored whenever L >= 2 (not in the children-expansion variant): the 4 rows of a level-1 entry
+    // together when p = 4 (rows4_score), else row by row
+    constexpr bool kRows4 = kScore == 1 && P == 4;
 #pragma unroll
     for (int g1 = 0; g1 < TB / P; ++g1) {
       float up[8], dn[8];
+      double part[4];
 #pragma unroll
       for (int c = 0; c < P; ++c) {
         float xf[8];
         unpack8(raw_s[(g1 * P + c) * kPoolThreads], xf);
-        if (kScore == 1) {  // level 0 is scored whenever L >= 2 (not in the children-expansion variant)
+        if (kRows4) {
+          part[c & 3] = lane_sq8(xf);
+        } else if (kScore == 1) {
           double x[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) x[i] = f64_of(xf[i]);
@@ -157,6 +193,11 @@ __device__ __forceinline__ void pool_score_body(const PoolJob& job, unsigned blo
           up[i] = (c == 0) ? xf[i] : add_up(up[i], xf[i]);
           dn[i] = (c == 0) ? xf[i] : add_dn(dn[i], xf[i]);
         }
+      }
+      if constexpr (kRows4) {  // the entry's 4 level-0 scores: lanes 0..3 of a row group hold one row each
+        float sc;
+        const int row = rows4_score<G>(part, lane, sc);
+        if (active && lane < 4) scores[dm.soff[0] + (int64_t)blk * W + t0 + g1 * P + row] = sc;
       }
       bool exact = true;
 #pragma unroll
@@ -239,7 +280,7 @@ __device__ __forceinline__ void pool_score_body(const PoolJob& job, unsigned blo
 // scored job's blocks are bound by instruction issue, the others by memory, and they overlap.  kScore is the scored
 // job's mode (jobs without a score array run the unscored body).
 template <int D, int P, int L, int kScore>
-__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(PoolJobs jobs, int njobs, LhDims dm) {
+__global__ void __launch_bounds__(kPoolThreads, 2) pool_score_kernel(PoolJobs jobs, int njobs, LhDims dm) {
   const int ji = (int)(blockIdx.x % (unsigned)njobs);
   const unsigned block = blockIdx.x / (unsigned)njobs;
   if (kScore != 0 && jobs.job[ji].scores != nullptr)
